@@ -61,6 +61,7 @@ extern "C" {
 #define SMLA_ERR_DEVICE (-2)    /* current device is not sm_100 (B200 class) */
 #define SMLA_ERR_CUDA (-3)      /* a CUDA runtime call failed */
 #define SMLA_ERR_LAUNCH (-4)    /* kernel launch failed */
+#define SMLA_ERR_SCRATCH (-5)   /* smla_decode_noalloc: the call needs more than SMLA_STATIC_SCRATCH_BYTES */
 
 /* Bits of the device error word. */
 #define SMLA_FLAG_BAD_PAGE 0x1u  /* a block-table entry outside [0, num_pages) was met and masked */
@@ -154,6 +155,38 @@ int smla_read_error(void *workspace, void *stream, uint32_t *flags);
 int smla_debug_gather(const uint8_t *kv_cache, const int32_t *block_table, const int32_t *topk_idx,
                       const int32_t *seq_lens, int B, int topk, int max_blocks, int num_pages, float *latents,
                       int32_t *page_slot, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * smla_decode_noalloc -- smla_decode for callers that cannot allocate device
+ * memory.  (No counterpart on the source pages: this is a library-usage addition.)
+ *
+ * Who needs it: a serving engine that has frozen its device memory pool after
+ * capturing its decode step into CUDA graphs, or a plugin host that owns every
+ * device allocation, cannot give this library a workspace.  This entry point
+ * takes the same arguments as smla_decode minus the workspace and uses instead
+ * a scratch array of SMLA_STATIC_SCRATCH_BYTES (32 MiB) that is part of the
+ * library's device image: every GPU that loads the library holds those bytes
+ * until the process exits.  It allocates and frees nothing (no cudaMalloc, no
+ * allocating library call).
+ *
+ *   - Limit: calls whose split-K partials need more than the array (header +
+ *     B*64*nsplit*(512+1)*4 bytes with the built-in split count) return
+ *     SMLA_ERR_SCRATCH without launching.  On a 148-SM B200 the built-in split
+ *     count keeps every call under 20 MB.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it has to start at zero (every partial is written before it is
+ *     read), but calls whose kernels overlap on the GPU (for example calls on
+ *     two streams of one device) race on it: serialise them.
+ *   - Device-side error flags land in the array's error word and are not
+ *     reported; use smla_decode with a workspace to read them.
+ */
+#define SMLA_STATIC_SCRATCH_BYTES (32u << 20)
+int smla_decode_noalloc(const void *q, const uint8_t *kv_cache, const int32_t *block_table, const int32_t *topk_idx,
+                        const int32_t *seq_lens, float sm_scale, float *out, float *lse, int B, int H, int topk,
+                        int max_blocks, int num_pages, void *stream);
 
 /* Build identification string (static storage). */
 const char *smla_version(void);

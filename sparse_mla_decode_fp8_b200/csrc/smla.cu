@@ -701,3 +701,47 @@ int smla_debug_gather(const uint8_t *kv_cache, const int32_t *block_table, const
 }
 
 }  // extern "C"
+
+// ======================================================================== no-allocation entry point
+// Some callers cannot hand the library a workspace: a serving engine that has
+// frozen its device memory pool after capturing its decode step into CUDA
+// graphs, or a plugin host that owns every device allocation and forbids its
+// plugins to call the allocator.  smla_decode_noalloc serves them from a
+// fixed scratch array that is part of this library's device image.
+namespace {
+
+constexpr size_t kStaticScratchBytes = SMLA_STATIC_SCRATCH_BYTES;
+void *g_static_scratch[kMaxDevices] = {};
+
+}  // namespace
+
+// Split-K partials and the error word of smla_decode_noalloc.  Every device that
+// loads this library holds these bytes until the process exits.  In host code
+// this name is only a stand-in: the device address comes from
+// cudaGetSymbolAddress, taken once per device below.
+static __device__ __align__(256) uint8_t g_smla_static_scratch[kStaticScratchBytes];
+
+extern "C" int smla_decode_noalloc(const void *q, const uint8_t *kv_cache, const int32_t *block_table,
+                                   const int32_t *topk_idx, const int32_t *seq_lens, float sm_scale, float *out,
+                                   float *lse, int B, int H, int topk, int max_blocks, int num_pages, void *stream) {
+    if (!sizes_ok(B, H, topk)) return SMLA_ERR_INVALID;
+    DeviceInfo *info = nullptr;
+    const int rc = device_info(info);
+    if (rc != SMLA_OK) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SMLA_ERR_CUDA;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_static_scratch[dev] == nullptr) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_smla_static_scratch) != cudaSuccess || p == nullptr) return SMLA_ERR_CUDA;
+            g_static_scratch[dev] = p;
+        }
+        scratch = g_static_scratch[dev];
+    }
+    if (workspace_for(B, topk, heuristic_splits(B, topk, info->sms)) > kStaticScratchBytes) return SMLA_ERR_SCRATCH;
+    return smla_decode_ex(q, kv_cache, block_table, topk_idx, seq_lens, sm_scale, out, lse, B, H, topk, max_blocks,
+                          num_pages, scratch, kStaticScratchBytes, nullptr, stream);
+}
+
