@@ -25,7 +25,9 @@
 //     a few large latents dominate).
 //   * The epilogue reads O^T from tensor memory and writes O/l (or a normalised
 //     split partial) and LSE = (m + log2 l) ln 2.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -39,30 +41,42 @@
 
 namespace smla {
 
-constexpr int kThreads = 256;
-constexpr int kTile = 128;
+constexpr int kTile = 128;           // topk slots per MMA tile (the M of S^T)
+constexpr int kThreads = 512;        // 16 warps, one CTA per SM; every warp takes part in every phase
+constexpr int kGatherThreads = 256;  // threads of the gather debug kernel
 
 // Dynamic shared memory map (bytes from a 1024-aligned base).
-constexpr int kSmemQ = 0;                           // 64 KB: 8 K-blocks x [64 heads x 128 B]
-constexpr int kSmemKV = kSmemQ + 65536;             // 128 KB: 8 K-blocks x [128 tokens x 128 B]
-constexpr int kSmemPhi = kSmemKV + 131072;          // 16 KB: [128 tokens x 64 heads] bf16
-constexpr int kSmemPlo = kSmemPhi + 16384;          // 16 KB
-constexpr int kSmemCodes = kSmemPlo + 16384;        // 128 int32 token codes
-constexpr int kSmemScales = kSmemCodes + 512;       // 128 x 8 B scale rows; reused as [4][64] f32
-constexpr int kSmemHeadM = kSmemScales + 1024;      // per-head running max (log2 units)
-constexpr int kSmemHeadL = kSmemHeadM + 256;        // per-head running sum
-constexpr int kSmemHeadAlpha = kSmemHeadL + 256;    // per-head rescale factor of this tile
-constexpr int kSmemHeadMnew = kSmemHeadAlpha + 256;  // per-head max after this tile
-constexpr int kSmemBar = kSmemHeadMnew + 256;       // mbarrier: MMA completion
-constexpr int kSmemBarSpare = kSmemBar + 8;         // mbarrier: test hook
-constexpr int kSmemTmemSlot = kSmemBarSpare + 8;
-constexpr int kSmemBytes = kSmemTmemSlot + 16;
+constexpr int kSmemQ = 0;                          // 64 KB: 8 K-blocks x [64 heads x 128 B], TMA-written
+constexpr int kSmemKV = kSmemQ + 65536;            // 128 KB: 8 K-blocks x [128 tokens x 128 B]
+constexpr int kSmemPhi = kSmemKV + 131072;         // 16 KB: P_hi^T [128 tokens x 64 heads] bf16
+constexpr int kSmemPlo = kSmemPhi + 16384;         // 16 KB: P_lo^T
+constexpr int kSmemCodes = kSmemPlo + 16384;       // [2][128] int32 token codes (double-buffered)
+constexpr int kSmemHeadM = kSmemCodes + 1024;      // [64] running max per head (log2 units)
+constexpr int kSmemHeadAlpha = kSmemHeadM + 256;   // [64] rescale factor of the last max update
+constexpr int kSmemRed = kSmemHeadAlpha + 256;     // [4][64] f32 cross-quadrant reduction scratch
+constexpr int kSmemBars = kSmemRed + 1024;         // mbarriers (8 B each)
+constexpr int kNumBars = 8;
+constexpr int kSmemTmemSlot = kSmemBars + kNumBars * 8;
+constexpr int kSmemAbort = kSmemTmemSlot + 4;
+constexpr int kSmemBytes = kSmemAbort + 12;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory limit");
 
-constexpr uint32_t kTmemCols = 512;  // O^T: columns [0,256), S^T: [256,320)
+enum Bar : int {
+    kBarQ = 0,       // Q landed (TMA transaction bytes)
+    kBarKvFull = 1,  // bf16 tile written (16 warp arrivals + st.async transaction bytes)
+    kBarSFull = 2,   // S^T complete (MMA commit)
+    kBarPFull = 3,   // P^T written (16 warp arrivals + st.async transaction bytes)
+    kBarPvDone = 4,  // PV complete (MMA commit): tile buffers and O^T free
+    kBarDrain = 5,   // final commit before tensor memory is released
+    kBarSpare = 6,   // test hook target
+};
+
+constexpr uint32_t kTmemCols = 512;  // O^T [0,256), S^T [256,320), per-lane running sums [320,384)
 constexpr uint32_t kTmemS = 256;
+constexpr uint32_t kTmemL = 320;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, true, true);
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(s - m) stays below 256 without a rescale
 
 struct DecodeParams {
     const uint16_t *q;
@@ -83,52 +97,290 @@ struct DecodeParams {
     int tiles_per_split;
     float scale_log2;  // sm_scale * log2(e)
     uint32_t debug_flags;
+    int cluster_merge;  // 1: the nsplit CTAs of a request form a cluster and merge through DSMEM
 };
 
-struct MaxOp {
-    __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
-};
-struct AddOp {
-    __device__ __forceinline__ float operator()(float a, float b) const { return a + b; }
-};
-
-// Reduces 64 per-thread values across the 32 lanes of a warp, value i with value
-// i of every other lane.  Afterwards lane L holds the results for entries 2L and
-// 2L+1 in v[0], v[1].  Each round halves the live entries: a lane keeps the half
-// selected by its lane bit and sends the other half to its partner.
-template <class Op>
-__device__ __forceinline__ void warp_transpose_reduce64(float (&v)[64], int lane, Op op) {
+// Reduces 16 per-thread values across the 32 lanes of a warp, value i with value i
+// of every other lane.  Afterwards lanes 2j and 2j+1 both hold the result for entry
+// j.  Each round halves the live entries: a lane keeps the half selected by its
+// lane bit and sends the other half to its partner; the last round combines pairs.
+template <bool kMax>
+__device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16], int lane) {
 #pragma unroll
-    for (int w = 32, off = 16; off >= 1; w >>= 1, off >>= 1) {
+    for (int w = 8, off = 16; off >= 2; w >>= 1, off >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < w; ++i) {
             const float send = upper ? v[i] : v[i + w];
             const float keep = upper ? v[i + w] : v[i];
-            v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, off));
+            const float got = __shfl_xor_sync(0xffffffffu, send, off);
+            v[i] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    const float got = __shfl_xor_sync(0xffffffffu, v[0], 1);
+    return kMax ? fmaxf(v[0], got) : v[0] + got;
+}
+
+// Bounded wait on an mbarrier phase.  Gives up when another thread has aborted the
+// CTA or when `timeout_ns` passes (then it aborts the CTA and flags the error).
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                           const DecodeParams &p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > p.timeout_ns) {
+            *abort_flag = 1;
+            atomicOr(p.err, SMLA_FLAG_TIMEOUT);
+            return false;
         }
     }
 }
 
-// Stores one 16-byte chunk of a token row, dequantised, into the swizzled tile.
-// c < 28: nope dims [16c, 16c+16) -> K-block c/4, chunks 2(c%4), 2(c%4)+1.
-// c >= 28: rope dims [448 + 8(c-28), +8) -> K-block 7, chunk c-28, copied as is.
-__device__ __forceinline__ void store_chunk(uint8_t *kv, int r, int c, const uint4 raw, const uint2 sc) {
-    const int sw = r & 7;
-    if (c < kNopeChunks) {
-        uint4 lo, hi;
-        dequant16(raw, scale_byte(sc, c >> 2), lo, hi);
-        uint8_t *row = kv + (c >> 2) * (kTile * 128) + r * 128;
-        const int oc = (c & 3) * 2;
-        *reinterpret_cast<uint4 *>(row + ((oc ^ sw) << 4)) = lo;
-        *reinterpret_cast<uint4 *>(row + (((oc + 1) ^ sw) << 4)) = hi;
+// Warp-uniform version: lane 0 waits, the verdict is broadcast, and every lane then
+// observes the completed phase itself (acquire) before touching the guarded data.
+__device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                const DecodeParams &p, int lane) {
+    int ok = 1;
+    if (lane == 0) ok = wait_phase(bar, parity, abort_flag, p) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) (void)mbar_try_wait(bar, parity);
+    return ok != 0;
+}
+
+// ------------------------------------------------------------------ gather + dequant
+// The 128 x 36 sixteen-byte chunks of a tile are dealt out in four groups, one per
+// K-block pair c (dims [128c, 128c+128)):
+//   pairs 0..2: 128 tokens x 8 nope chunks (16 dims)          -> 2 items per thread
+//   pair 3:     128 tokens x (4 nope + 8 rope chunks)          -> 3 items per thread
+// Consecutive threads take consecutive chunks of a token row (coalesced loads).
+template <int C>
+struct PairShape {
+    static constexpr int kItems = (C < 3) ? 2 : 3;
+};
+
+template <int C>
+__device__ __forceinline__ void pair_item(int t, int u, int &r, int &chunk, int &kb, int &oc, bool &nope) {
+    const int j = t + kThreads * u;
+    if constexpr (C < 3) {
+        r = j >> 3;
+        const int k = j & 7;
+        chunk = 8 * C + k;
+        kb = 2 * C + (k >> 2);
+        oc = 2 * (k & 3);
+        nope = true;
     } else {
-        uint8_t *row = kv + 7 * (kTile * 128) + r * 128;
-        *reinterpret_cast<uint4 *>(row + (((c - kNopeChunks) ^ sw) << 4)) = raw;
+        r = j / 12;
+        const int k = j - 12 * r;
+        if (k < 4) {
+            chunk = 24 + k;
+            kb = 6;
+            oc = 2 * k;
+            nope = true;
+        } else {
+            chunk = 28 + (k - 4);
+            kb = 7;
+            oc = k - 4;
+            nope = false;
+        }
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+// The FP8 bytes (and the scale byte) of one tile, held in registers between the
+// load and the dequantisation.
+struct TileRegs {
+    uint4 raw0[2], raw1[2], raw2[2], raw3[3];
+    uint32_t sc0[2], sc1[2], sc2[2], sc3[3];
+};
+
+template <int C>
+__device__ __forceinline__ void load_pair(int t, const int *codes, const uint8_t *cache,
+                                          uint4 (&raw)[PairShape<C>::kItems], uint32_t (&sc)[PairShape<C>::kItems]) {
+#pragma unroll
+    for (int u = 0; u < PairShape<C>::kItems; ++u) {
+        int r, chunk, kb, oc;
+        bool nope;
+        pair_item<C>(t, u, r, chunk, kb, oc, nope);
+        const int code = codes[r];
+        raw[u] = make_uint4(0u, 0u, 0u, 0u);
+        sc[u] = 0u;
+        if (code >= 0) {
+            raw[u] = ld_stream_v4(token_row(cache, code) + chunk * 16);
+            if (nope) sc[u] = ld_stream_u8(token_scales(cache, code) + (chunk >> 2));
+        }
+    }
+}
+
+__device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t *cache, TileRegs &tr) {
+    load_pair<0>(t, codes, cache, tr.raw0, tr.sc0);
+    load_pair<1>(t, codes, cache, tr.raw1, tr.sc1);
+    load_pair<2>(t, codes, cache, tr.raw2, tr.sc2);
+    load_pair<3>(t, codes, cache, tr.raw3, tr.sc3);
+}
+
+// Dequantises this thread's items of pair C into the swizzled bf16 tile with st.async
+// (async proxy, completing transaction bytes on `bar`).  Returns the bytes stored.
+template <int C>
+__device__ __forceinline__ uint32_t store_pair(int t, uint32_t kv, uint32_t bar,
+                                               const uint4 (&raw)[PairShape<C>::kItems],
+                                               const uint32_t (&sc)[PairShape<C>::kItems]) {
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int u = 0; u < PairShape<C>::kItems; ++u) {
+        int r, chunk, kb, oc;
+        bool nope;
+        pair_item<C>(t, u, r, chunk, kb, oc, nope);
+        const uint32_t row = kv + kb * (kTile * 128) + r * 128;
+        const int sw = r & 7;
+        if (nope) {
+            uint4 lo, hi;
+            dequant16(raw[u], sc[u], lo, hi);
+            // odd K-blocks store their high half first so the 8 lanes of a store phase hit 8 bank groups
+            if ((kb & 1) == 0) {
+                st_async_v4(row + ((oc ^ sw) << 4), lo, bar);
+                st_async_v4(row + (((oc + 1) ^ sw) << 4), hi, bar);
+            } else {
+                st_async_v4(row + (((oc + 1) ^ sw) << 4), hi, bar);
+                st_async_v4(row + ((oc ^ sw) << 4), lo, bar);
+            }
+            bytes += 32;
+        } else {
+            st_async_v4(row + ((oc ^ sw) << 4), raw[u], bar);
+            bytes += 16;
+        }
+    }
+    return bytes;
+}
+
+template <int C>
+__device__ __forceinline__ uint32_t pair_bytes(int t) {
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int u = 0; u < PairShape<C>::kItems; ++u) {
+        int r, chunk, kb, oc;
+        bool nope;
+        pair_item<C>(t, u, r, chunk, kb, oc, nope);
+        bytes += nope ? 32u : 16u;
+    }
+    return bytes;
+}
+
+// ------------------------------------------------------------------ split merge in a cluster
+// The nsplit CTAs of one request form a thread-block cluster.  After the last PV,
+// every CTA holds un-normalised O^T_s (tensor memory), its per-head running max m_s
+// and sum l_s.  With L = log2 sum_s 2^(m_s) l_s, the merged output is
+// O = sum_s 2^(m_s - L) O^T_s (the split-K log-sum-exp merge), LSE = L ln 2.
+// Output dims are dealt out by 128-dim chunk: chunk mc belongs to CTA mc % nsplit.
+// Exchange (distributed shared memory, after every CTA's MMAs are done):
+//   (m_s, l_s) -> every CTA's P^T region; raw O^T chunks -> the owner's Q/KV region,
+//   one 128 x 64 fp32 block per (owned chunk, sender), rows padded to 272 bytes.
+constexpr int kRecvRow = 272;
+constexpr int kRecvBlock = 128 * kRecvRow;
+
+__device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool ok, int n, int tid, int q, int g,
+                                              int lane, uint32_t tmem, uint32_t lane_base, uint8_t *smem,
+                                              const float *head_m, float *head_l2, const float *l_head) {
+    const int ns = p.nsplit;
+    const int me = static_cast<int>(cluster_ctarank());
+    float *exch = reinterpret_cast<float *>(smem + kSmemPhi);  // [s][m(64) | l(64)]
+    uint8_t *recv = smem + kSmemQ;                              // Q and KV tiles are dead here
+    const int d = 32 * q + lane;                                // row of O^T within a chunk
+    // barrier 1: every CTA's MMAs are done, so remote writes into its operand buffers are safe
+    cluster_sync();
+    if (ok) {
+        if (tid < kHeads)
+            for (int s = 0; s < ns; ++s) {
+                st_cluster_f32(map_to_rank(exch + me * 128 + tid, s), head_m[tid]);
+                st_cluster_f32(map_to_rank(exch + me * 128 + 64 + tid, s), l_head[tid]);
+            }
+#pragma unroll 1
+        for (int mc = 0; mc < 4; ++mc) {
+            const int owner = mc % ns;
+            if (owner == me) continue;
+            const int slot = (me < owner) ? me : me - 1;
+            const uint8_t *dst = recv + ((mc / ns) * (ns - 1) + slot) * kRecvBlock + d * kRecvRow + 64 * g;
+            float o[16];
+            tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, o);
+            tmem_wait_ld();
+            const uint32_t raddr = map_to_rank(dst, owner);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st_cluster_v4(raddr + 16 * j, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        }
+    }
+    // barrier 2: all exchanged values have landed
+    cluster_sync();
+    if (!ok) return;
+    if (tid < kHeads) {
+        float mx = -INFINITY;
+        for (int s = 0; s < ns; ++s)
+            if (exch[s * 128 + 64 + tid] > 0.0f) mx = fmaxf(mx, exch[s * 128 + tid]);
+        float sum = 0.0f;
+        for (int s = 0; s < ns; ++s) {
+            const float l = exch[s * 128 + 64 + tid];
+            if (l > 0.0f) sum += exp2f(exch[s * 128 + tid] - mx) * l;
+        }
+        const float L = (sum > 0.0f) ? mx + log2f(sum) : -INFINITY;
+        head_l2[tid] = L;
+        if (me == 0)
+            p.lse[static_cast<size_t>(b) * kHeads + tid] = (sum > 0.0f) ? L * 0.69314718055994531f : -INFINITY;
+    }
+    __syncthreads();
+    if (tid < kHeads) {
+        const float L = head_l2[tid];
+        for (int s = 0; s < ns; ++s) {
+            const float l = exch[s * 128 + 64 + tid];
+            exch[s * 128 + tid] = (l > 0.0f && L != -INFINITY) ? exp2f(exch[s * 128 + tid] - L) : 0.0f;
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int mc = me; mc < 4; mc += ns) {
+        const int lci = mc / ns;
+        float acc[16];
+        if (n > 0) {
+            tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, acc);
+            tmem_wait_ld();
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) acc[h] = (n > 0) ? acc[h] * exch[me * 128 + 16 * g + h] : 0.0f;
+        for (int s = 0; s < ns; ++s) {
+            if (s == me) continue;
+            const int slot = (s < me) ? s : s - 1;
+            const float4 *src =
+                reinterpret_cast<const float4 *>(recv + (lci * (ns - 1) + slot) * kRecvBlock + d * kRecvRow + 64 * g);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = src[j];
+                acc[4 * j] += v.x * exch[s * 128 + 16 * g + 4 * j];
+                acc[4 * j + 1] += v.y * exch[s * 128 + 16 * g + 4 * j + 1];
+                acc[4 * j + 2] += v.z * exch[s * 128 + 16 * g + 4 * j + 2];
+                acc[4 * j + 3] += v.w * exch[s * 128 + 16 * g + 4 * j + 3];
+            }
+        }
+        float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * g) * kDim + 128 * mc + d;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) dst[h * kDim] = acc[h];
+    }
+}
+
+// ------------------------------------------------------------------ the decode kernel
+// One CTA per (topk split, request), 16 warps, one 128-slot tile at a time:
+//   1. every thread dequantises its 9 prefetched chunks of the tile into the bf16
+//      tile (st.async, completion counted on one mbarrier);
+//   2. every thread issues the loads of the next tile (they stay in flight through
+//      the MMA and softmax phases), and threads 0..127 run the index translation of
+//      the tile after next, spread over the phases so its latency is hidden;
+//   3. thread 0 issues S^T = K.Q^T (32 tcgen05.mma, M=128 tokens, N=64 heads);
+//   4. softmax on all 16 warps: warp w reads TMEM lanes 32(w%4).. (tokens) and
+//      columns 16(w/4).. (heads); p = 2^(s*c - m) against the running max m, which
+//      is raised (with a rescale of O^T and of the per-lane running sums) only when a
+//      score exceeds it by more than 2^8; P^T is written as bf16 hi + lo terms;
+//   5. thread 0 issues O^T += V^T.P_hi^T + V^T.P_lo^T (64 tcgen05.mma).
+// The epilogue reduces the per-lane sums and writes O/l and LSE, merging the splits of
+// a request inside its thread-block cluster when there are several.
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_q) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -145,264 +397,303 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     uint8_t *sPhi = smem + kSmemPhi;
     uint8_t *sPlo = smem + kSmemPlo;
     int *codes = reinterpret_cast<int *>(smem + kSmemCodes);
-    uint2 *scales = reinterpret_cast<uint2 *>(smem + kSmemScales);
-    float *red = reinterpret_cast<float *>(smem + kSmemScales);
     float *head_m = reinterpret_cast<float *>(smem + kSmemHeadM);
-    float *head_l = reinterpret_cast<float *>(smem + kSmemHeadL);
     float *head_alpha = reinterpret_cast<float *>(smem + kSmemHeadAlpha);
-    float *head_mnew = reinterpret_cast<float *>(smem + kSmemHeadMnew);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kSmemBar);
-    uint64_t *bar_spare = reinterpret_cast<uint64_t *>(smem + kSmemBarSpare);
+    float *red = reinterpret_cast<float *>(smem + kSmemRed);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBars);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmemTmemSlot);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmemAbort);
+
+    const int num_tiles = (p.topk + kTile - 1) / kTile;
+    const int t_begin = split * p.tiles_per_split;
+    const int n = max(0, min(num_tiles, t_begin + p.tiles_per_split) - t_begin);
+    const int seq_len = __ldg(p.seq_lens + b);
+    const int32_t *bt_row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+    const int32_t *idx_row = p.topk_idx + static_cast<size_t>(b) * p.topk;
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        mbar_init(bar_spare, 1);
+    if (tid == 32) {
+        mbar_init(&bars[kBarQ], 1);
+        mbar_init(&bars[kBarKvFull], 16);
+        mbar_init(&bars[kBarSFull], 1);
+        mbar_init(&bars[kBarPFull], 16);
+        mbar_init(&bars[kBarPvDone], 1);
+        mbar_init(&bars[kBarDrain], 1);
+        mbar_init(&bars[kBarSpare], 1);
         fence_barrier_init();
+        *abort_flag = 0;
     }
-    if (tid < kHeads) {
-        head_m[tid] = -INFINITY;
-        head_l[tid] = 0.0f;
+    if (tid < kHeads) head_m[tid] = -INFINITY;
+    // index translation of tiles 0 and 1 (threads 0..255: tile tid/128, slot tid%128)
+    if (tid < 2 * kTile) {
+        const int ti = tid >> 7;
+        const int slot = (t_begin + ti) * kTile + (tid & (kTile - 1));
+        int code = -1;
+        if (ti < n && slot < p.topk)
+            code = translate_slot(bt_row, p.max_blocks, seq_len, p.num_pages, __ldg(idx_row + slot), p.err);
+        codes[tid] = code;
     }
-    // Q[b] -> shared memory, K-major 128-byte swizzle: K-block kb = dims [64kb, 64kb+64).
-    {
-        const uint4 *qg = reinterpret_cast<const uint4 *>(p.q + static_cast<size_t>(b) * kHeads * kDim);
-#pragma unroll 4
-        for (int c = tid; c < kHeads * kDim / 8; c += kThreads) {
-            const int head = c >> 6, kc = c & 63;
-            const uint4 v = ld_stream_v4(qg + c);
-            *reinterpret_cast<uint4 *>(sQ + (kc >> 3) * 8192 + head * 128 + (((kc & 7) ^ (head & 7)) << 4)) = v;
-        }
-    }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t sQ_a = smem_addr(sQ), sKV_a = smem_addr(sKV), sPhi_a = smem_addr(sPhi), sPlo_a = smem_addr(sPlo);
+    const uint32_t me = cluster_ctarank();
+    const uint32_t kv_c = map_to_rank(sKV, me);
+    const uint32_t phi_c = map_to_rank(sPhi, me);
+    const uint32_t plo_c = map_to_rank(sPlo, me);
+    const uint32_t bar_kv_c = map_to_rank(&bars[kBarKvFull], me);
+    const uint32_t bar_p_c = map_to_rank(&bars[kBarPFull], me);
 
-    const int num_tiles = (p.topk + kTile - 1) / kTile;
-    const int t_begin = split * p.tiles_per_split;
-    const int t_end = min(num_tiles, t_begin + p.tiles_per_split);
-    const int seq_len = __ldg(p.seq_lens + b);
-    const int32_t *bt_row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-    const int32_t *idx_row = p.topk_idx + static_cast<size_t>(b) * p.topk;
-    const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
-
-    uint32_t phase = 0;
-    bool have_o = false, failed = false, first = true, spare_armed = false;
-
-    for (int t = t_begin; t < t_end; ++t) {
-        // ---- translate 128 slots, fetch their scale rows
-        int code = -1;
-        if (tid < kTile) {
-            const int i = t * kTile + tid;
-            if (i < p.topk) code = translate_slot(bt_row, p.max_blocks, seq_len, p.num_pages, __ldg(idx_row + i), p.err);
-            codes[tid] = code;
-            scales[tid] = (code >= 0) ? ld_stream_v2(token_scales(p.cache, code)) : make_uint2(0u, 0u);
-        }
-        if (__syncthreads_count(code >= 0) == 0) continue;  // whole tile masked: nothing to add
-
-        // ---- gather + dequantise 128 x 36 chunks into the bf16 tile
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
 #pragma unroll
-        for (int it = 0; it < kTile * kRowChunks / kThreads; it += 6) {
-            uint4 raw[6];
-            int rr[6], cc[6];
-#pragma unroll
-            for (int u = 0; u < 6; ++u) {
-                const int i = tid + (it + u) * kThreads;
-                rr[u] = i / kRowChunks;
-                cc[u] = i - rr[u] * kRowChunks;
-                const int cd = codes[rr[u]];
-                raw[u] = (cd >= 0) ? ld_stream_v4(token_row(p.cache, cd) + cc[u] * 16) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int u = 0; u < 6; ++u) store_chunk(sKV, rr[u], cc[u], raw[u], scales[rr[u]]);
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---- S^T = K_tile . Q^T  (M=128 tokens, N=64 heads, K=512)
-        const bool skip_commit = first && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
-        if (tid == 0) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int kb = 0; kb < 8; ++kb) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = sw128_desc(sKV_a + kb * (kTile * 128) + kk * 32, 16, 1024);
-                    const uint64_t bq = sw128_desc(sQ_a + kb * 8192 + kk * 32, 16, 1024);
-                    mma_bf16_ss(tmem + kTmemS, a, bq, kIdescQK, (kb | kk) != 0);
-                }
-            }
-            mma_commit(skip_commit ? bar_spare : bar);
-        }
-        if (skip_commit) spare_armed = true;
-        first = false;
-        bool ok = mbar_wait(bar, phase, p.timeout_ns);
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        phase ^= 1u;
-        tc_fence_after_sync();
-
-        // ---- online softmax (warps 0-3: thread = token lane of S^T)
-        if (warp < 4) {
-            const int r = tid;
-            const bool valid = codes[r] >= 0;
-            float v[64];
-            tmem_ld64(tmem + lane_base + kTmemS, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 64; ++h) v[h] = valid ? v[h] * p.scale_log2 : -INFINITY;
-            warp_transpose_reduce64(v, lane, MaxOp());
-            red[warp * 64 + 2 * lane] = v[0];
-            red[warp * 64 + 2 * lane + 1] = v[1];
-            named_barrier_sync(1, 128);
-            if (r < kHeads) {
-                const float tm = fmaxf(fmaxf(red[r], red[64 + r]), fmaxf(red[128 + r], red[192 + r]));
-                const float mo = head_m[r];
-                const float mn = fmaxf(mo, tm);
-                head_alpha[r] = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
-                head_mnew[r] = mn;
-            }
-            named_barrier_sync(1, 128);
-            tmem_ld64(tmem + lane_base + kTmemS, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h4 = 0; h4 < 16; ++h4) {
-                const float4 mn = reinterpret_cast<const float4 *>(head_mnew)[h4];
-                const float m4[4] = {mn.x, mn.y, mn.z, mn.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int h = 4 * h4 + j;
-                    v[h] = (valid && m4[j] != -INFINITY) ? exp2f(v[h] * p.scale_log2 - m4[j]) : 0.0f;
-                }
-            }
-            // P^T rows (token r, 64 heads) as bf16 hi and lo terms, MN-major swizzled.
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float a0 = v[8 * c + 2 * j], a1 = v[8 * c + 2 * j + 1];
-                    const __nv_bfloat162 hb = __floats2bfloat162_rn(a0, a1);
-                    const float2 hf = __bfloat1622float2(hb);
-                    const __nv_bfloat162 lb = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
-                    hw[j] = *reinterpret_cast<const uint32_t *>(&hb);
-                    lw[j] = *reinterpret_cast<const uint32_t *>(&lb);
-                }
-                const int off = r * 128 + ((c ^ (r & 7)) << 4);
-                *reinterpret_cast<uint4 *>(sPhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(sPlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
-            warp_transpose_reduce64(v, lane, AddOp());
-            red[warp * 64 + 2 * lane] = v[0];
-            red[warp * 64 + 2 * lane + 1] = v[1];
-            named_barrier_sync(1, 128);
-            if (r < kHeads) {
-                const float s = (red[r] + red[64 + r]) + (red[128 + r] + red[192 + r]);
-                head_l[r] = head_l[r] * head_alpha[r] + s;
-                head_m[r] = head_mnew[r];
-            }
-            if (have_o) {
-                float alpha[64];
-                bool any = false;
-#pragma unroll
-                for (int h4 = 0; h4 < 16; ++h4) {
-                    const float4 a4 = reinterpret_cast<const float4 *>(head_alpha)[h4];
-                    alpha[4 * h4] = a4.x;
-                    alpha[4 * h4 + 1] = a4.y;
-                    alpha[4 * h4 + 2] = a4.z;
-                    alpha[4 * h4 + 3] = a4.w;
-                    any |= (a4.x != 1.0f) | (a4.y != 1.0f) | (a4.z != 1.0f) | (a4.w != 1.0f);
-                }
-                if (any) {
-#pragma unroll 1
-                    for (int mc = 0; mc < 4; ++mc) {
-                        float o[64];
-                        tmem_ld64(tmem + lane_base + 64 * mc, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int h = 0; h < 64; ++h) o[h] *= alpha[h];
-                        tmem_st64(tmem + lane_base + 64 * mc, o);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-        }
-        __syncthreads();
-
-        // ---- O^T += V^T . P^T  (4 x M=128 dims, N=64 heads, K=128 tokens; P = hi + lo)
-        if (tid == 0) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int mc = 0; mc < 4; ++mc) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t a = sw128_desc(sKV_a + 2 * mc * (kTile * 128) + ks * 2048, kTile * 128, 1024);
-                    const uint64_t bh = sw128_desc(sPhi_a + ks * 2048, 8192, 1024);
-                    const uint64_t bl = sw128_desc(sPlo_a + ks * 2048, 8192, 1024);
-                    mma_bf16_ss(tmem + 64 * mc, a, bh, kIdescPV, (have_o || ks > 0) ? 1u : 0u);
-                    mma_bf16_ss(tmem + 64 * mc, a, bl, kIdescPV, 1u);
-                }
-            }
-            mma_commit(bar);
-        }
-        ok = mbar_wait(bar, phase, p.timeout_ns);
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        phase ^= 1u;
-        tc_fence_after_sync();
-        have_o = true;
+        for (int kb = 0; kb < 8; ++kb) tma_load_2d(sQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
     }
 
-    if (failed) {
+    // thread roles inside the softmax / epilogue: TMEM lane quadrant q, head group g
+    const int q = warp & 3;
+    const int g = warp >> 2;
+    const int r = 32 * q + lane;  // token lane of S^T, output-dim lane of O^T
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const float c = p.scale_log2;
+    const uint32_t warp_tile_bytes = [&] {
+        const uint32_t v = pair_bytes<0>(tid) + pair_bytes<1>(tid) + pair_bytes<2>(tid) + pair_bytes<3>(tid);
+        return __reduce_add_sync(0xffffffffu, v);
+    }();
+
+    // MMA descriptors of the operand bases; every MMA adds a compile-time offset (bytes >> 4)
+    const uint64_t dQK_a = sw128_desc(smem_addr(sKV), 16, 1024);
+    const uint64_t dQK_b = sw128_desc(smem_addr(sQ), 16, 1024);
+    const uint64_t dPV_a = sw128_desc(smem_addr(sKV), kTile * 128, 1024);
+    const uint64_t dPV_bh = sw128_desc(smem_addr(sPhi), 8192, 1024);
+    const uint64_t dPV_bl = sw128_desc(smem_addr(sPlo), 8192, 1024);
+
+    TileRegs tr;
+    if (n > 0) load_tile(tid, codes, p.cache, tr);
+    bool failed = false, spare_used = false;
+    int idx_next = -1, page_next = -1;
+
+    for (int i = 0; i < n; ++i) {
+        const int buf = i & 1;
+        const bool valid = codes[buf * kTile + r] >= 0;
+        // ---- 1. dequantise the tile
+        if (lane == 0) mbar_arrive_expect_tx(&bars[kBarKvFull], warp_tile_bytes);
+        __syncwarp();
+        store_pair<0>(tid, kv_c, bar_kv_c, tr.raw0, tr.sc0);
+        store_pair<1>(tid, kv_c, bar_kv_c, tr.raw1, tr.sc1);
+        store_pair<2>(tid, kv_c, bar_kv_c, tr.raw2, tr.sc2);
+        store_pair<3>(tid, kv_c, bar_kv_c, tr.raw3, tr.sc3);
+        // ---- 2. prefetch the next tile, start translating the tile after it
+        if (i + 1 < n) load_tile(tid, codes + (buf ^ 1) * kTile, p.cache, tr);
+        const int slot2 = (t_begin + i + 2) * kTile + tid;
+        if (tid < kTile && i + 2 < n && slot2 < p.topk) idx_next = __ldg(idx_row + slot2);
+        // ---- 3. S^T = K.Q^T
         if (tid == 0) {
-            atomicOr(p.err, SMLA_FLAG_TIMEOUT);
-            // MMAs committed to the spare barrier must finish before tensor memory is released.
-            if (spare_armed) (void)mbar_wait(bar_spare, 0, p.timeout_ns);
-        }
-    } else if (warp < 4) {
-        // ---- epilogue: O^T lane = output dim within a 128-row block, column = head
-        float inv_l[64];
+            bool ok = (i > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
+                      wait_phase(&bars[kBarKvFull], i & 1, abort_flag, p);
+            if (ok) {
+                tc_fence_after_sync();
 #pragma unroll
-        for (int h = 0; h < 64; ++h) {
-            const float l = head_l[h];
-            inv_l[h] = (have_o && l > 0.0f) ? 1.0f / l : 0.0f;
-        }
-#pragma unroll 1
-        for (int mc = 0; mc < 4; ++mc) {
-            float o[64];
-            tmem_ld64(tmem + lane_base + 64 * mc, o);
-            tmem_wait_ld();
-            const int d = 128 * mc + 32 * warp + lane;
-            if (p.nsplit == 1) {
-                float *dst = p.out + static_cast<size_t>(b) * kHeads * kDim + d;
+                for (int kb = 0; kb < 8; ++kb)
 #pragma unroll
-                for (int h = 0; h < 64; ++h) dst[h * kDim] = o[h] * inv_l[h];
-            } else {
-                float *dst = p.part_o + (static_cast<size_t>(b) * kHeads * p.nsplit + split) * kDim + d;
-#pragma unroll
-                for (int h = 0; h < 64; ++h) dst[static_cast<size_t>(h) * p.nsplit * kDim] = o[h] * inv_l[h];
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + kTmemS, dQK_a + (kb * (kTile * 128) + kk * 32) / 16,
+                                    dQK_b + (kb * 8192 + kk * 32) / 16, kIdescQK, (kb | kk) != 0);
+                const bool hook = (i == 0) && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
+                mma_commit(hook ? &bars[kBarSpare] : &bars[kBarSFull]);
+                spare_used = hook;
             }
         }
+        bool ok = warp_wait_phase(&bars[kBarSFull], i & 1, abort_flag, p, lane);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after_sync();
+        if (tid < kTile && i + 2 < n && idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks)
+            page_next = __ldg(bt_row + (idx_next >> 8));
+        // ---- 4. online softmax over 16 warps
+        float x[16];
+        tmem_ld16(tmem + lane_base + kTmemS + 16 * g, x);
+        tmem_wait_ld();
+        bool over = false;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            x[h] = valid ? fmaf(x[h], c, -head_m[16 * g + h]) : -INFINITY;
+            over |= x[h] > kRescaleThreshold;
+        }
+        if (__syncthreads_or(over)) {
+            // raise each head's running max to max(m, tile max); rescale what was accumulated
+            tmem_ld16(tmem + lane_base + kTmemS + 16 * g, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h) x[h] = valid ? x[h] * c : -INFINITY;
+            const float tmax = warp_transpose_reduce16<true>(x, lane);
+            if ((lane & 1) == 0) red[q * 64 + 16 * g + (lane >> 1)] = tmax;
+            __syncthreads();
+            if (tid < kHeads) {
+                const float tm = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
+                const float mo = head_m[tid];
+                const float mn = fmaxf(mo, tm);
+                head_alpha[tid] = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+                head_m[tid] = mn;
+            }
+            __syncthreads();
+            if (i > 0) {
+                float al[16], o[16];
+#pragma unroll
+                for (int h = 0; h < 16; ++h) al[h] = head_alpha[16 * g + h];
+#pragma unroll 1
+                for (int cc = 0; cc < 5; ++cc) {  // 4 O^T chunks + the running sums
+                    const uint32_t col = (cc < 4 ? 64u * cc : kTmemL) + 16u * g;
+                    tmem_ld16(tmem + lane_base + col, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) o[h] *= al[h];
+                    tmem_st16(tmem + lane_base + col, o);
+                }
+            }
+            tmem_ld16(tmem + lane_base + kTmemS + 16 * g, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h) x[h] = valid ? fmaf(x[h], c, -head_m[16 * g + h]) : -INFINITY;
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) x[h] = fast_exp2(x[h]);
+        {
+            float l[16];
+            if (i == 0) {
+#pragma unroll
+                for (int h = 0; h < 16; ++h) l[h] = x[h];
+            } else {
+                tmem_ld16(tmem + lane_base + kTmemL + 16 * g, l);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 16; ++h) l[h] += x[h];
+            }
+            tmem_st16(tmem + lane_base + kTmemL + 16 * g, l);
+        }
+        // P^T row r, heads 16g..16g+15: two 16-byte chunks of hi and two of lo
+        if (lane == 0) mbar_arrive_expect_tx(&bars[kBarPFull], 32 * 64);
+        __syncwarp();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float a0 = x[8 * half + 2 * j], a1 = x[8 * half + 2 * j + 1];
+                hw[j] = pack_bf16x2(a0, a1);
+                lw[j] = pack_bf16x2(a0 - __uint_as_float(hw[j] << 16), a1 - __uint_as_float(hw[j] & 0xFFFF0000u));
+            }
+            const uint32_t off = r * 128 + (((2 * g + half) ^ (r & 7)) << 4);
+            st_async_v4(phi_c + off, make_uint4(hw[0], hw[1], hw[2], hw[3]), bar_p_c);
+            st_async_v4(plo_c + off, make_uint4(lw[0], lw[1], lw[2], lw[3]), bar_p_c);
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncthreads();
+        // ---- 5. O^T += V^T.P^T
+        if (tid == 0) {
+            if (wait_phase(&bars[kBarPFull], i & 1, abort_flag, p)) {
+                tc_fence_after_sync();
+                const uint32_t acc0 = (i > 0) ? 1u : 0u;
+#pragma unroll
+                for (int mc = 0; mc < 4; ++mc) {
+                    const uint64_t a0 = dPV_a + static_cast<uint64_t>(mc * 2 * (kTile * 128 / 16));
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bh + ks * (2048 / 16), kIdescPV,
+                                    ks > 0 ? 1u : acc0);
+                        mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bl + ks * (2048 / 16), kIdescPV, 1u);
+                    }
+                }
+                mma_commit(&bars[kBarPvDone]);
+            }
+        }
+        ok = warp_wait_phase(&bars[kBarPvDone], i & 1, abort_flag, p, lane);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after_sync();
+        // translation of tile i+2 completes into the buffer tile i used
+        if (tid < kTile && i + 2 < n) {
+            int code = -1;
+            if (idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks) {
+                if (page_next < 0 || static_cast<long long>(page_next) >= p.num_pages)
+                    atomicOr(p.err, SMLA_FLAG_BAD_PAGE);
+                else
+                    code = page_next * kPageTokens + (idx_next & (kPageTokens - 1));
+            }
+            codes[buf * kTile + tid] = code;
+            idx_next = -1;
+            page_next = -1;
+        }
+        __syncthreads();
+    }
+
+    // every MMA issued above must be complete before tensor memory is released
+    if (tid == 0) {
+        if (spare_used) (void)mbar_wait(&bars[kBarSpare], 0, p.timeout_ns);
+        mma_commit(&bars[kBarDrain]);
+        (void)mbar_wait(&bars[kBarDrain], 0, p.timeout_ns);
+    }
+    __syncthreads();
+    const bool ok = !failed && !*abort_flag;
+
+    // ---- epilogue: per-head sums over the 128 token lanes, then O/l (or the cluster merge)
+    float l_part = 0.0f;
+    if (ok && n > 0) {
+        tc_fence_after_sync();
+        float v[16];
+        tmem_ld16(tmem + lane_base + kTmemL + 16 * g, v);
+        tmem_wait_ld();
+        l_part = warp_transpose_reduce16<false>(v, lane);
+    }
+    if ((lane & 1) == 0) red[q * 64 + 16 * g + (lane >> 1)] = l_part;
+    __syncthreads();
+    float *l_head = head_alpha;  // per-head sums for the epilogue
+    if (tid < kHeads) l_head[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
+    __syncthreads();
+    if (p.cluster_merge) {
+        float *l2 = red;  // scratch for L (the cross-quadrant values are consumed)
+        cluster_epilogue(p, b, ok, n, tid, q, g, lane, tmem, lane_base, smem, head_m, l2, l_head);
+    } else if (ok) {
         if (tid < kHeads) {
-            const float l = head_l[tid];
-            const float val = (have_o && l > 0.0f) ? (head_m[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            const float l = l_head[tid];
+            const float val = (l > 0.0f) ? (head_m[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
             if (p.nsplit == 1)
                 p.lse[static_cast<size_t>(b) * kHeads + tid] = val;
             else
                 p.part_lse[(static_cast<size_t>(b) * kHeads + tid) * p.nsplit + split] = val;
+        }
+        float inv[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            const float l = l_head[16 * g + h];
+            inv[h] = (l > 0.0f) ? 1.0f / l : 0.0f;
+        }
+#pragma unroll 1
+        for (int mc = 0; mc < 4; ++mc) {
+            float o[16];
+            if (n > 0) {
+                tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, o);
+                tmem_wait_ld();
+            }
+            const int d = 128 * mc + r;
+            if (p.nsplit == 1) {
+                float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * g) * kDim + d;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) dst[h * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
+            } else {
+                float *dst = p.part_o + ((static_cast<size_t>(b) * kHeads + 16 * g) * p.nsplit + split) * kDim + d;
+#pragma unroll
+                for (int h = 0; h < 16; ++h)
+                    dst[static_cast<size_t>(h) * p.nsplit * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
+            }
         }
     }
     tc_fence_before_sync();
@@ -451,13 +742,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
 
 // Gather debug kernel: the translation and dequantisation of decode_kernel,
 // written out as fp32 latents and (page, slot) pairs.  Grid (tiles, B).
-__global__ void __launch_bounds__(kThreads) gather_kernel(const uint8_t *cache, const int32_t *block_table,
+__global__ void __launch_bounds__(kGatherThreads) gather_kernel(const uint8_t *cache, const int32_t *block_table,
                                                           const int32_t *topk_idx, const int32_t *seq_lens,
                                                           long long num_pages, int topk, int max_blocks,
                                                           float *latents, int32_t *page_slot, uint32_t *err) {
     __shared__ int codes[kTile];
     __shared__ uint2 scales[kTile];
-    __shared__ __align__(16) uint8_t tile_row[kThreads][32];
+    __shared__ __align__(16) uint8_t tile_row[kGatherThreads][32];
     const int tid = threadIdx.x, t = blockIdx.x, b = blockIdx.y;
     if (tid < kTile) {
         const int i = t * kTile + tid;
@@ -473,7 +764,7 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint8_t *cache, 
         }
     }
     __syncthreads();
-    for (int i = tid; i < kTile * kRowChunks; i += kThreads) {
+    for (int i = tid; i < kTile * kRowChunks; i += kGatherThreads) {
         const int r = i / kRowChunks, c = i - r * kRowChunks;
         const int slot = t * kTile + r;
         if (slot >= topk) continue;
@@ -514,6 +805,38 @@ struct DeviceInfo {
 
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000 &fn) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_encode_tiled == nullptr) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || f == nullptr)
+            return SMLA_ERR_CUDA;
+        g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    fn = g_encode_tiled;
+    return SMLA_OK;
+}
+
+// Q [B*64 rows, 512 bf16] as a 2-D tensor; a box of 64 dims x 64 heads with the
+// 128-byte swizzle lands as one K-block of the shared-memory Q operand.
+int encode_q_map(CUtensorMap *map, const void *q, int B) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    const int rc = tensor_map_encoder(fn);
+    if (rc != SMLA_OK) return rc;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(SMLA_DIM), static_cast<cuuint64_t>(B) * SMLA_HEADS};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(SMLA_DIM) * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(q), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SMLA_OK : SMLA_ERR_INVALID;
+}
 
 int device_info(DeviceInfo *&info) {
     int dev = 0;
@@ -560,9 +883,14 @@ bool sizes_ok(int B, int H, int topk) {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Up to this many splits of a request merge inside a thread-block cluster (through
+// distributed shared memory); beyond it they go through global partials and the
+// merge kernel.
+constexpr int kMaxClusterSplits = 4;
+
 size_t workspace_for(int B, int topk, int nsplit) {
     size_t bytes = SMLA_WORKSPACE_HEADER;
-    if (nsplit > 1) {
+    if (nsplit > kMaxClusterSplits) {
         const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
         bytes += round256(rows * sizeof(float)) + rows * SMLA_DIM * sizeof(float);
     }
@@ -651,11 +979,28 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     p.scale_log2 = sm_scale * 1.4426950408889634f;
     p.debug_flags = opts ? opts->debug_flags : 0u;
 
+    alignas(64) CUtensorMap tmap_q;
+    rc = encode_q_map(&tmap_q, q, B);
+    if (rc != SMLA_OK) return rc;
+
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     (void)cudaGetLastError();
-    smla::decode_kernel<<<dim3(nsplit, B), smla::kThreads, smla::kSmemBytes, st>>>(p);
+    p.cluster_merge = (nsplit > 1 && nsplit <= kMaxClusterSplits) ? 1 : 0;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(nsplit, B);
+    cfg.blockDim = dim3(smla::kThreads);
+    cfg.dynamicSmemBytes = smla::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.cluster_merge ? nsplit : 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, smla::decode_kernel, p, tmap_q) != cudaSuccess) return SMLA_ERR_LAUNCH;
     if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_LAUNCH;
-    if (nsplit > 1) {
+    if (nsplit > 1 && !p.cluster_merge) {
         smla::combine_kernel<<<static_cast<unsigned>(B) * SMLA_HEADS, 128, 0, st>>>(p.part_o, p.part_lse, out, lse,
                                                                                    nsplit);
         if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_LAUNCH;
@@ -694,7 +1039,7 @@ int smla_debug_gather(const uint8_t *kv_cache, const int32_t *block_table, const
     const int rc = device_info(info);
     if (rc != SMLA_OK) return rc;
     (void)cudaGetLastError();
-    smla::gather_kernel<<<dim3(num_tiles(topk), B), smla::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+    smla::gather_kernel<<<dim3(num_tiles(topk), B), smla::kGatherThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         kv_cache, block_table, topk_idx, seq_lens, num_pages, topk, max_blocks, latents, page_slot,
         static_cast<uint32_t *>(workspace));
     return cudaGetLastError() == cudaSuccess ? SMLA_OK : SMLA_ERR_LAUNCH;
