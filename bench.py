@@ -239,8 +239,6 @@ def run_cuda(args):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
-    ncall = 200
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ncall)]
     with ClockSampler(dev.index) as clk:
         with torch.cuda.stream(stream):
             # clocks under load before the timed region (graph replays for about a second)
@@ -252,15 +250,9 @@ def run_cuda(args):
             for _ in range(reps):
                 g.replay()
             e1.record(stream)
-            # per-launch durations: events around single calls (eager, so the GPU runs one call at a time)
-            for i in range(ncall):
-                evs[i][0].record(stream)
-                step(i, stream)
-                evs[i][1].record(stream)
         stream.synchronize()
     barrier()
     elapsed_ms = e0.elapsed_time(e1)
-    per_call_ms = float(np.median([a.elapsed_time(b) for a, b in evs]))
     t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
     if dist is not None:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -320,7 +312,11 @@ def run_cuda(args):
     ms_step = max_ms / steps
     units = W.roofline_units(w.replica(0))
     peaks, peak_src = load_peaks()
-    call_ms = per_call_ms
+    # up to kMaxClusterSplits splits merge inside the decode kernel's cluster: one launch per call;
+    # beyond that a second (combine) kernel follows
+    launches_per_call = 1 if nsplit <= 4 else 2
+    # this rank's own average duration of one decode launch over the timed region (graph replays on `stream`)
+    call_ms = elapsed_ms / steps
     achieved_gbs = units["bytes"] / (call_ms * 1e-3) / 1e9
     achieved_tf = units["flops"] / (call_ms * 1e-3) / 1e12
     t_hbm_us = units["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
@@ -350,9 +346,10 @@ def run_cuda(args):
                      "roofline_us": max(t_hbm_us, t_tc_us), "frac_of_roofline": max(t_hbm_us, t_tc_us) / (call_ms * 1e3),
                      "tc_tflops": achieved_tf, "tc_peak_tflops": peaks["bf16_tflops"],
                      "tc_frac": achieved_tf / peaks["bf16_tflops"],
-                     "per_launch": "median of 200 single calls bracketed by CUDA events" +
-                     (" (decode + split-K merge kernels)" if nsplit > 1 else "")},
-        "gpu_launches": steps * (1 if nsplit == 1 else 2),
+                     "per_launch": "CUDA events around the timed graph replays on the launching stream, "
+                     f"divided by {steps} calls" + (" (decode + combine kernels)" if launches_per_call > 1 else
+                                                    " (one decode kernel per call)")},
+        "gpu_launches": steps * launches_per_call,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

@@ -9,7 +9,7 @@
 // run on tensor cores with fp32 accumulation, and split partials are merged by
 // their log-sum-exp (Step 5).
 //
-// B200 mapping, per CTA (one per SM, 256 threads):
+// B200 mapping, per CTA (one per SM, 512 threads):
 //   * Q[b] (64 heads x 512, bf16) stays in shared memory for the whole CTA.
 //   * A tile of 128 topk slots is translated through the block table, its FP8
 //     rows are loaded with 16-byte loads and dequantised in registers into a
@@ -59,16 +59,18 @@ constexpr int kNumBars = 8;
 constexpr int kSmemTmemSlot = kSmemBars + kNumBars * 8;
 constexpr int kSmemAbort = kSmemTmemSlot + 4;
 constexpr int kSmemBytes = kSmemAbort + 12;
+constexpr int kSmemMl = kSmemCodes - 2048;         // cluster merge: [4][m(64) | l(64)] f32, inside P_lo (dead by then)
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory limit");
 
 enum Bar : int {
     kBarQ = 0,       // Q landed (TMA transaction bytes)
-    kBarKvFull = 1,  // bf16 tile written (16 warp arrivals + st.async transaction bytes)
+    kBarKvFull = 1,  // bf16 tile written (16 warp arrivals after a proxy fence)
     kBarSFull = 2,   // S^T complete (MMA commit)
-    kBarPFull = 3,   // P^T written (16 warp arrivals + st.async transaction bytes)
+    kBarPFull = 3,   // P^T written (16 warp arrivals after a proxy fence)
     kBarPvDone = 4,  // PV complete (MMA commit): tile buffers and O^T free
     kBarDrain = 5,   // final commit before tensor memory is released
     kBarSpare = 6,   // test hook target
+    kBarRecv = 7,    // cluster merge: partials received from the other CTAs (bulk-copy bytes)
 };
 
 constexpr uint32_t kTmemCols = 512;  // O^T [0,256), S^T [256,320), per-lane running sums [320,384)
@@ -219,13 +221,11 @@ __device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t
     load_pair<3>(t, codes, cache, tr.raw3, tr.sc3);
 }
 
-// Dequantises this thread's items of pair C into the swizzled bf16 tile with st.async
-// (async proxy, completing transaction bytes on `bar`).  Returns the bytes stored.
+// Dequantises this thread's items of pair C into the swizzled bf16 tile (plain shared
+// stores; `kv` is the tile's shared-window address).
 template <int C>
-__device__ __forceinline__ uint32_t store_pair(int t, uint32_t kv, uint32_t bar,
-                                               const uint4 (&raw)[PairShape<C>::kItems],
-                                               const uint32_t (&sc)[PairShape<C>::kItems]) {
-    uint32_t bytes = 0;
+__device__ __forceinline__ void store_pair(int t, uint32_t kv, const uint4 (&raw)[PairShape<C>::kItems],
+                                           const uint32_t (&sc)[PairShape<C>::kItems]) {
 #pragma unroll
     for (int u = 0; u < PairShape<C>::kItems; ++u) {
         int r, chunk, kb, oc;
@@ -238,136 +238,165 @@ __device__ __forceinline__ uint32_t store_pair(int t, uint32_t kv, uint32_t bar,
             dequant16(raw[u], sc[u], lo, hi);
             // odd K-blocks store their high half first so the 8 lanes of a store phase hit 8 bank groups
             if ((kb & 1) == 0) {
-                st_async_v4(row + ((oc ^ sw) << 4), lo, bar);
-                st_async_v4(row + (((oc + 1) ^ sw) << 4), hi, bar);
+                sts_v4(row + ((oc ^ sw) << 4), lo);
+                sts_v4(row + (((oc + 1) ^ sw) << 4), hi);
             } else {
-                st_async_v4(row + (((oc + 1) ^ sw) << 4), hi, bar);
-                st_async_v4(row + ((oc ^ sw) << 4), lo, bar);
+                sts_v4(row + (((oc + 1) ^ sw) << 4), hi);
+                sts_v4(row + ((oc ^ sw) << 4), lo);
             }
-            bytes += 32;
         } else {
-            st_async_v4(row + ((oc ^ sw) << 4), raw[u], bar);
-            bytes += 16;
+            sts_v4(row + ((oc ^ sw) << 4), raw[u]);
         }
     }
-    return bytes;
-}
-
-template <int C>
-__device__ __forceinline__ uint32_t pair_bytes(int t) {
-    uint32_t bytes = 0;
-#pragma unroll
-    for (int u = 0; u < PairShape<C>::kItems; ++u) {
-        int r, chunk, kb, oc;
-        bool nope;
-        pair_item<C>(t, u, r, chunk, kb, oc, nope);
-        bytes += nope ? 32u : 16u;
-    }
-    return bytes;
 }
 
 // ------------------------------------------------------------------ split merge in a cluster
 // The nsplit CTAs of one request form a thread-block cluster.  After the last PV,
-// every CTA holds un-normalised O^T_s (tensor memory), its per-head running max m_s
-// and sum l_s.  With L = log2 sum_s 2^(m_s) l_s, the merged output is
-// O = sum_s 2^(m_s - L) O^T_s (the split-K log-sum-exp merge), LSE = L ln 2.
+// CTA s holds un-normalised O^T_s (tensor memory), its per-head running max m_s (log2
+// units) and sum l_s.  With L = log2 sum_s 2^(m_s) l_s, the merged output is
+// O = sum_s 2^(m_s - L) O^T_s and LSE = L ln 2 (the split-K log-sum-exp merge).
 // Output dims are dealt out by 128-dim chunk: chunk mc belongs to CTA mc % nsplit.
-// Exchange (distributed shared memory, after every CTA's MMAs are done):
-//   (m_s, l_s) -> every CTA's P^T region; raw O^T chunks -> the owner's Q/KV region,
-//   one 128 x 64 fp32 block per (owned chunk, sender), rows padded to 272 bytes.
-constexpr int kRecvRow = 272;
-constexpr int kRecvBlock = 128 * kRecvRow;
+// Once every CTA's MMAs are done (its Q, KV and P buffers are dead), each CTA stages
+// its (m_s, l_s) row and the O^T_s chunks it does not own in its own shared memory
+// and sends them with bulk shared-to-shared copies into the owners' receive areas,
+// where they are counted in bytes on kBarRecv.  Receive area of a CTA: blocks
+// [owned chunk lci][sender slot] from offset 0, the (m, l) rows at kSmemMl; its send
+// staging follows its receive blocks.
+constexpr int kRecvRow = 272;               // 64 heads x fp32 + 16 B pad: conflict-free row stores
+constexpr int kRecvBlock = 128 * kRecvRow;  // one 128-dim chunk of O^T
+constexpr int kMlRow = 512;                 // m[64] | l[64], f32
+
+__host__ __device__ constexpr int owned_chunks(int me, int ns) { return (4 - me + ns - 1) / ns; }
+static_assert(4 * kRecvBlock + 2 * kRecvBlock <= kSmemMl, "receive + send areas overlap the (m, l) rows");
+static_assert(3 * kRecvBlock + 3 * kRecvBlock <= kSmemMl, "receive + send areas overlap the (m, l) rows");
 
 __device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool ok, int n, int tid, int q, int g,
                                               int lane, uint32_t tmem, uint32_t lane_base, uint8_t *smem,
-                                              const float *head_m, float *head_l2, const float *l_head) {
+                                              uint64_t *bar_recv, const float *head_m, const float *l_head,
+                                              float *weights) {
     const int ns = p.nsplit;
     const int me = static_cast<int>(cluster_ctarank());
-    float *exch = reinterpret_cast<float *>(smem + kSmemPhi);  // [s][m(64) | l(64)]
-    uint8_t *recv = smem + kSmemQ;                              // Q and KV tiles are dead here
-    const int d = 32 * q + lane;                                // row of O^T within a chunk
-    // barrier 1: every CTA's MMAs are done, so remote writes into its operand buffers are safe
+    const int n_own = owned_chunks(me, ns);
+    const uint32_t base = smem_addr(smem);
+    const uint32_t send = base + n_own * (ns - 1) * kRecvBlock;
+    float *ml = reinterpret_cast<float *>(smem + kSmemMl);  // [s][m(64) | l(64)]
+    const int d = 32 * q + lane;                            // row of O^T within a chunk
+    const bool live = ok && n > 0;
+
+    // barrier 1: every CTA's MMAs are done, so its operand buffers may be overwritten
     cluster_sync();
-    if (ok) {
-        if (tid < kHeads)
-            for (int s = 0; s < ns; ++s) {
-                st_cluster_f32(map_to_rank(exch + me * 128 + tid, s), head_m[tid]);
-                st_cluster_f32(map_to_rank(exch + me * 128 + 64 + tid, s), l_head[tid]);
-            }
+    if (tid < kHeads) {
+        ml[me * 128 + tid] = live ? head_m[tid] : -INFINITY;
+        ml[me * 128 + 64 + tid] = live ? l_head[tid] : 0.0f;
+    }
+    {
+        int js = 0;
 #pragma unroll 1
+        for (int mc = 0; mc < 4; ++mc) {
+            if (mc % ns == me) continue;
+            float o[16];
+            if (live) {
+                tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int h = 0; h < 16; ++h) o[h] = 0.0f;
+            }
+            const uint32_t row = send + js * kRecvBlock + d * kRecvRow + 64 * g;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sts_v4f(row + 16 * j, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            ++js;
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid < ns && tid != me) {
+        const int peer = tid;
+        const uint32_t bar_c = map_to_rank(bar_recv, peer);
+        bulk_copy_to_cluster(map_to_rank(ml + me * 128, peer), smem_addr(ml + me * 128), kMlRow, bar_c);
+        int js = 0;
         for (int mc = 0; mc < 4; ++mc) {
             const int owner = mc % ns;
             if (owner == me) continue;
-            const int slot = (me < owner) ? me : me - 1;
-            const uint8_t *dst = recv + ((mc / ns) * (ns - 1) + slot) * kRecvBlock + d * kRecvRow + 64 * g;
-            float o[16];
-            tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, o);
-            tmem_wait_ld();
-            const uint32_t raddr = map_to_rank(dst, owner);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) st_cluster_v4(raddr + 16 * j, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            if (owner == peer) {
+                const int slot = (me < peer) ? me : me - 1;
+                const int blk = (mc / ns) * (ns - 1) + slot;
+                bulk_copy_to_cluster(map_to_rank(smem + blk * kRecvBlock, peer), send + js * kRecvBlock, kRecvBlock,
+                                     bar_c);
+            }
+            ++js;
         }
     }
-    // barrier 2: all exchanged values have landed
-    cluster_sync();
-    if (!ok) return;
+    // the other CTAs' rows and chunks have landed (bounded wait; the copies are in flight
+    // whatever happened elsewhere, so the abort flag does not cut it short)
+    int got = 1;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_recv, (ns - 1) * (kMlRow + n_own * kRecvBlock));
+        got = mbar_wait(bar_recv, 0, p.timeout_ns) ? 1 : 0;
+        if (!got) atomicOr(p.err, SMLA_FLAG_TIMEOUT);
+    }
+    got = __syncthreads_and(got);
+    if (got) (void)mbar_try_wait(bar_recv, 0);  // every thread observes the completed phase
+    const bool write = got && ok;
     if (tid < kHeads) {
         float mx = -INFINITY;
         for (int s = 0; s < ns; ++s)
-            if (exch[s * 128 + 64 + tid] > 0.0f) mx = fmaxf(mx, exch[s * 128 + tid]);
+            if (ml[s * 128 + 64 + tid] > 0.0f) mx = fmaxf(mx, ml[s * 128 + tid]);
         float sum = 0.0f;
         for (int s = 0; s < ns; ++s) {
-            const float l = exch[s * 128 + 64 + tid];
-            if (l > 0.0f) sum += exp2f(exch[s * 128 + tid] - mx) * l;
+            const float l = ml[s * 128 + 64 + tid];
+            if (l > 0.0f) sum += exp2f(ml[s * 128 + tid] - mx) * l;
         }
         const float L = (sum > 0.0f) ? mx + log2f(sum) : -INFINITY;
-        head_l2[tid] = L;
-        if (me == 0)
+        for (int s = 0; s < ns; ++s)
+            weights[s * kHeads + tid] = (sum > 0.0f && ml[s * 128 + 64 + tid] > 0.0f) ? exp2f(ml[s * 128 + tid] - L)
+                                                                                      : 0.0f;
+        if (me == 0 && write)
             p.lse[static_cast<size_t>(b) * kHeads + tid] = (sum > 0.0f) ? L * 0.69314718055994531f : -INFINITY;
     }
     __syncthreads();
-    if (tid < kHeads) {
-        const float L = head_l2[tid];
-        for (int s = 0; s < ns; ++s) {
-            const float l = exch[s * 128 + 64 + tid];
-            exch[s * 128 + tid] = (l > 0.0f && L != -INFINITY) ? exp2f(exch[s * 128 + tid] - L) : 0.0f;
-        }
-    }
-    __syncthreads();
+    if (write) {
 #pragma unroll 1
-    for (int mc = me; mc < 4; mc += ns) {
-        const int lci = mc / ns;
-        float acc[16];
-        if (n > 0) {
-            tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, acc);
-            tmem_wait_ld();
-        }
-#pragma unroll
-        for (int h = 0; h < 16; ++h) acc[h] = (n > 0) ? acc[h] * exch[me * 128 + 16 * g + h] : 0.0f;
-        for (int s = 0; s < ns; ++s) {
-            if (s == me) continue;
-            const int slot = (s < me) ? s : s - 1;
-            const float4 *src =
-                reinterpret_cast<const float4 *>(recv + (lci * (ns - 1) + slot) * kRecvBlock + d * kRecvRow + 64 * g);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float4 v = src[j];
-                acc[4 * j] += v.x * exch[s * 128 + 16 * g + 4 * j];
-                acc[4 * j + 1] += v.y * exch[s * 128 + 16 * g + 4 * j + 1];
-                acc[4 * j + 2] += v.z * exch[s * 128 + 16 * g + 4 * j + 2];
-                acc[4 * j + 3] += v.w * exch[s * 128 + 16 * g + 4 * j + 3];
+        for (int mc = me; mc < 4; mc += ns) {
+            const int lci = mc / ns;
+            float acc[16];
+            if (live) {
+                tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, acc);
+                tmem_wait_ld();
             }
-        }
-        float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * g) * kDim + 128 * mc + d;
 #pragma unroll
-        for (int h = 0; h < 16; ++h) dst[h * kDim] = acc[h];
+            for (int h = 0; h < 16; ++h) {
+                const float w = weights[me * kHeads + 16 * g + h];
+                acc[h] = (live && w != 0.0f) ? acc[h] * w : 0.0f;
+            }
+            for (int s = 0; s < ns; ++s) {
+                if (s == me) continue;
+                const int slot = (s < me) ? s : s - 1;
+                const float4 *src = reinterpret_cast<const float4 *>(smem + (lci * (ns - 1) + slot) * kRecvBlock +
+                                                                     d * kRecvRow + 64 * g);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 v = src[j];
+                    const float *w = weights + s * kHeads + 16 * g + 4 * j;
+                    if (w[0] != 0.0f) acc[4 * j] += v.x * w[0];
+                    if (w[1] != 0.0f) acc[4 * j + 1] += v.y * w[1];
+                    if (w[2] != 0.0f) acc[4 * j + 2] += v.z * w[2];
+                    if (w[3] != 0.0f) acc[4 * j + 3] += v.w * w[3];
+                }
+            }
+            float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * g) * kDim + 128 * mc + d;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) dst[h * kDim] = acc[h];
+        }
     }
+    // barrier 2: no CTA leaves while a bulk copy may still be reading its staging area
+    cluster_sync();
 }
 
 // ------------------------------------------------------------------ the decode kernel
 // One CTA per (topk split, request), 16 warps, one 128-slot tile at a time:
 //   1. every thread dequantises its 9 prefetched chunks of the tile into the bf16
-//      tile (st.async, completion counted on one mbarrier);
+//      tile (plain shared stores, a proxy fence, one mbarrier arrival per warp);
 //   2. every thread issues the loads of the next tile (they stay in flight through
 //      the MMA and softmax phases), and threads 0..127 run the index translation of
 //      the tile after next, spread over the phases so its latency is hidden;
@@ -423,8 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars[kBarPvDone], 1);
         mbar_init(&bars[kBarDrain], 1);
         mbar_init(&bars[kBarSpare], 1);
+        mbar_init(&bars[kBarRecv], 1);
         fence_barrier_init();
         *abort_flag = 0;
+        mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) tma_load_2d(sQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
     }
     if (tid < kHeads) head_m[tid] = -INFINITY;
     // index translation of tiles 0 and 1 (threads 0..255: tile tid/128, slot tid%128)
@@ -440,18 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t me = cluster_ctarank();
-    const uint32_t kv_c = map_to_rank(sKV, me);
-    const uint32_t phi_c = map_to_rank(sPhi, me);
-    const uint32_t plo_c = map_to_rank(sPlo, me);
-    const uint32_t bar_kv_c = map_to_rank(&bars[kBarKvFull], me);
-    const uint32_t bar_p_c = map_to_rank(&bars[kBarPFull], me);
-
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
-#pragma unroll
-        for (int kb = 0; kb < 8; ++kb) tma_load_2d(sQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
-    }
+    const uint32_t kv_s = smem_addr(sKV);
+    const uint32_t phi_s = smem_addr(sPhi);
+    const uint32_t plo_s = smem_addr(sPlo);
 
     // thread roles inside the softmax / epilogue: TMEM lane quadrant q, head group g
     const int q = warp & 3;
@@ -459,10 +483,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = 32 * q + lane;  // token lane of S^T, output-dim lane of O^T
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const float c = p.scale_log2;
-    const uint32_t warp_tile_bytes = [&] {
-        const uint32_t v = pair_bytes<0>(tid) + pair_bytes<1>(tid) + pair_bytes<2>(tid) + pair_bytes<3>(tid);
-        return __reduce_add_sync(0xffffffffu, v);
-    }();
 
     // MMA descriptors of the operand bases; every MMA adds a compile-time offset (bytes >> 4)
     const uint64_t dQK_a = sw128_desc(smem_addr(sKV), 16, 1024);
@@ -480,12 +500,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = i & 1;
         const bool valid = codes[buf * kTile + r] >= 0;
         // ---- 1. dequantise the tile
-        if (lane == 0) mbar_arrive_expect_tx(&bars[kBarKvFull], warp_tile_bytes);
+        store_pair<0>(tid, kv_s, tr.raw0, tr.sc0);
+        store_pair<1>(tid, kv_s, tr.raw1, tr.sc1);
+        store_pair<2>(tid, kv_s, tr.raw2, tr.sc2);
+        store_pair<3>(tid, kv_s, tr.raw3, tr.sc3);
+        fence_proxy_async_smem();  // this thread's tile stores -> visible to the tensor core
         __syncwarp();
-        store_pair<0>(tid, kv_c, bar_kv_c, tr.raw0, tr.sc0);
-        store_pair<1>(tid, kv_c, bar_kv_c, tr.raw1, tr.sc1);
-        store_pair<2>(tid, kv_c, bar_kv_c, tr.raw2, tr.sc2);
-        store_pair<3>(tid, kv_c, bar_kv_c, tr.raw3, tr.sc3);
+        if (lane == 0) mbar_arrive(&bars[kBarKvFull]);
         // ---- 2. prefetch the next tile, start translating the tile after it
         if (i + 1 < n) load_tile(tid, codes + (buf ^ 1) * kTile, p.cache, tr);
         const int slot2 = (t_begin + i + 2) * kTile + tid;
@@ -577,8 +598,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tmem + lane_base + kTmemL + 16 * g, l);
         }
         // P^T row r, heads 16g..16g+15: two 16-byte chunks of hi and two of lo
-        if (lane == 0) mbar_arrive_expect_tx(&bars[kBarPFull], 32 * 64);
-        __syncwarp();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             uint32_t hw[4], lw[4];
@@ -589,9 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lw[j] = pack_bf16x2(a0 - __uint_as_float(hw[j] << 16), a1 - __uint_as_float(hw[j] & 0xFFFF0000u));
             }
             const uint32_t off = r * 128 + (((2 * g + half) ^ (r & 7)) << 4);
-            st_async_v4(phi_c + off, make_uint4(hw[0], hw[1], hw[2], hw[3]), bar_p_c);
-            st_async_v4(plo_c + off, make_uint4(lw[0], lw[1], lw[2], lw[3]), bar_p_c);
+            sts_v4(phi_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+            sts_v4(plo_s + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarPFull]);
         tmem_wait_st();
         tc_fence_before_sync();
         __syncthreads();
@@ -659,8 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < kHeads) l_head[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
     __syncthreads();
     if (p.cluster_merge) {
-        float *l2 = red;  // scratch for L (the cross-quadrant values are consumed)
-        cluster_epilogue(p, b, ok, n, tid, q, g, lane, tmem, lane_base, smem, head_m, l2, l_head);
+        cluster_epilogue(p, b, ok, n, tid, q, g, lane, tmem, lane_base, smem, &bars[kBarRecv], head_m, l_head, red);
     } else if (ok) {
         if (tid < kHeads) {
             const float l = l_head[tid];
