@@ -104,10 +104,12 @@ typedef struct smla_options {
  *   workspace   device scratch of at least smla_workspace_bytes(B, H, topk)
  *               bytes, 256-byte aligned.  Its first 4 bytes are the sticky error
  *               word: zero it once (cudaMemset or smla_read_error) before first use.
- *               The rest holds split-K partials between the two kernels of a call;
+ *               The rest holds the split-K exchange of a call (partials between
+ *               the CTAs of a request, or between the decode and merge kernels);
  *               concurrent calls must not share a workspace.
- * Launches the decode kernel and, when the topk range is split, the combine
- * kernel, on `stream`.
+ * Launches the decode kernel on `stream`.  A request whose topk range is split
+ * in 2..4 parts is merged inside the kernel by the thread-block cluster of its
+ * parts; with more parts the combine kernel follows.
  */
 int smla_decode(const void *q, const uint8_t *kv_cache, const int32_t *block_table, const int32_t *topk_idx,
                 const int32_t *seq_lens, float sm_scale, float *out, float *lse, int B, int H, int topk,
@@ -169,8 +171,8 @@ int smla_debug_gather(const uint8_t *kv_cache, const int32_t *block_table, const
  * until the process exits.  It allocates and frees nothing (no cudaMalloc, no
  * allocating library call).
  *
- *   - Limit: calls whose split-K partials need more than the array (header +
- *     B*64*nsplit*(512+1)*4 bytes with the built-in split count) return
+ *   - Limit: calls whose split-K exchange needs more than the array (what
+ *     smla_workspace_bytes reports for the built-in split count) return
  *     SMLA_ERR_SCRATCH without launching.  On a 148-SM B200 the built-in split
  *     count keeps every call under 20 MB.
  *   - The first call on each device looks up the array's device address

@@ -254,6 +254,21 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int c0,
         : "memory");
 }
 
+// Untiled bulk copy (no multicast) of `bytes` from global memory into this CTA's shared
+// memory; both addresses 16-byte aligned, bytes a multiple of 16.  Completion is
+// signalled as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Orders this thread's generic-proxy memory writes before later async-proxy accesses
+// (bulk copies) that are ordered after it.
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+
 // Or-reduction of a predicate over the `nthreads` threads of named barrier `id`.
 __device__ __forceinline__ bool barrier_or(uint32_t id, uint32_t nthreads, bool pred) {
     uint32_t out;
@@ -308,18 +323,6 @@ __device__ __forceinline__ void sts_v4(uint32_t saddr, uint4 v) {
 }
 __device__ __forceinline__ void sts_v4f(uint32_t saddr, float a, float b, float c, float d) {
     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this
-// CTA's shared memory into the shared memory of a CTA of the cluster; completion is
-// counted in transaction bytes on that CTA's mbarrier.  No multicast.
-__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                     uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-        : "memory");
 }
 
 // Brings a kernel-parameter tensor map into the descriptor cache ahead of its first use.

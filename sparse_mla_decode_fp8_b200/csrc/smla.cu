@@ -9,22 +9,26 @@
 // run on tensor cores with fp32 accumulation, and split partials are merged by
 // their log-sum-exp (Step 5).
 //
-// B200 mapping, per CTA (one per SM, 512 threads):
-//   * Q[b] (64 heads x 512, bf16) stays in shared memory for the whole CTA.
-//   * A tile of 128 topk slots is translated through the block table, its FP8
-//     rows are loaded with 16-byte loads and dequantised in registers into a
-//     bf16 [128 x 512] tile in the 128-byte-swizzled layout the tensor core reads.
+// B200 mapping, per CTA (one per SM, 512 threads in two warp roles):
+//   * Q[b] (64 heads x 512, bf16) stays in shared memory for the whole CTA (TMA).
+//   * Producer warps translate a tile of 128 topk slots through the block table,
+//     keep its FP8 rows in flight in registers (16-byte loads) while the previous
+//     tile is computed, and dequantise them into a bf16 [128 x 512] tile in the
+//     128-byte-swizzled layout the tensor core reads, one 128-dim K-block pair at
+//     a time as the previous tile's PV releases it.
 //   * S^T[128 tokens x 64 heads] = K_tile . Q^T: tcgen05.mma M=128 N=64, fp32 in
-//     tensor memory.  Tokens fill the 128-row M dimension, not the 64 heads.
-//   * Softmax warps (one thread per token lane) read S^T from tensor memory,
-//     keep the running max / sum per head, rescale O^T in tensor memory when the
-//     max grows, and write P^T as two bf16 terms (P = P_hi + P_lo).
+//     tensor memory (two S^T buffers).  Tokens fill the 128-row M dimension, not
+//     the 64 heads.
+//   * Softmax warps (one thread per token lane and 32 heads) read S^T from tensor
+//     memory, keep the running max per head and the sums in registers, rescale
+//     O^T in tensor memory when the max grows, and write P^T as two bf16 terms
+//     (P = P_hi + P_lo).  One of their threads issues the MMAs.
 //   * O^T[512 x 64] += V^T . P^T with V = the same bf16 tile read MN-major:
 //     4 MMAs of M=128 per 16-token step, once with P_hi and once with P_lo, so P
 //     carries ~16 significant bits (a single bf16 P is not accurate enough when
 //     a few large latents dominate).
-//   * The epilogue reads O^T from tensor memory and writes O/l (or a normalised
-//     split partial) and LSE = (m + log2 l) ln 2.
+//   * The epilogue reads O^T from tensor memory and writes O/l (or merges the
+//     splits of a request inside its cluster) and LSE = (m + log2 l) ln 2.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -41,41 +45,50 @@
 
 namespace smla {
 
-constexpr int kTile = 128;           // topk slots per MMA tile (the M of S^T)
-constexpr int kThreads = 512;        // 16 warps, one CTA per SM; every warp takes part in every phase
-constexpr int kGatherThreads = 256;  // threads of the gather debug kernel
+constexpr int kTile = 128;                                  // topk slots per MMA tile (the M of S^T)
+constexpr int kSoftmaxWarps = 8;                            // warps 0..7: softmax and epilogue; warp 0 also
+                                                            // owns tensor memory and issues TMA and MMAs
+constexpr int kProducerWarps = 8;                           // warps 8..15: translation, gather, dequantisation
+constexpr int kThreads = 32 * (kSoftmaxWarps + kProducerWarps);  // 512: 128 registers per thread
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;         // 256
+constexpr int kProducerThreads = 32 * kProducerWarps;       // 256
+constexpr int kGatherThreads = 256;                         // threads of the gather debug kernel
+constexpr uint32_t kBarIdSoftmax = 1;                       // named barrier of the softmax warps
+constexpr uint32_t kBarIdProducer = 2;                      // named barrier of the producer warps
 
 // Dynamic shared memory map (bytes from a 1024-aligned base).
-constexpr int kSmemQ = 0;                          // 64 KB: 8 K-blocks x [64 heads x 128 B], TMA-written
-constexpr int kSmemKV = kSmemQ + 65536;            // 128 KB: 8 K-blocks x [128 tokens x 128 B]
-constexpr int kSmemPhi = kSmemKV + 131072;         // 16 KB: P_hi^T [128 tokens x 64 heads] bf16
-constexpr int kSmemPlo = kSmemPhi + 16384;         // 16 KB: P_lo^T
-constexpr int kSmemCodes = kSmemPlo + 16384;       // [2][128] int32 token codes (double-buffered)
-constexpr int kSmemHeadM = kSmemCodes + 1024;      // [64] running max per head (log2 units)
-constexpr int kSmemHeadAlpha = kSmemHeadM + 256;   // [64] rescale factor of the last max update
-constexpr int kSmemRed = kSmemHeadAlpha + 256;     // [4][64] f32 cross-quadrant reduction scratch
-constexpr int kSmemBars = kSmemRed + 1024;         // mbarriers (8 B each)
-constexpr int kNumBars = 8;
-constexpr int kSmemTmemSlot = kSmemBars + kNumBars * 8;
-constexpr int kSmemAbort = kSmemTmemSlot + 4;
-constexpr int kSmemBytes = kSmemAbort + 12;
-constexpr int kSmemMl = kSmemCodes - 2048;         // cluster merge: [4][m(64) | l(64)] f32, inside P_lo (dead by then)
-static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory limit");
+constexpr int kSmemQ = 0;                         // 64 KB: 8 K-blocks x [64 heads x 128 B], TMA-written
+constexpr int kSmemKV = kSmemQ + 65536;           // 128 KB: 8 K-blocks x [128 tokens x 128 B]
+constexpr int kSmemPhi = kSmemKV + 131072;        // 16 KB: P_hi^T [128 tokens x 64 heads] bf16
+constexpr int kSmemPlo = kSmemPhi + 16384;        // 16 KB: P_lo^T
+constexpr int kSmemCodes = kSmemPlo + 16384;      // [2][128] int32 token codes (producers only)
+constexpr int kSmemMask = kSmemCodes + 1024;      // [4][4] u32: valid-token bits of a tile, ring of 4 tiles
+constexpr int kSmemHeadM = kSmemMask + 64;        // [64] running max per head (log2 units)
+constexpr int kSmemHeadAlpha = kSmemHeadM + 256;  // [64] rescale factor of the last max update; then the sums
+constexpr int kSmemRed = kSmemHeadAlpha + 256;    // [4][64] f32 cross-quadrant scratch
+constexpr int kSmemBars = kSmemRed + 1024;        // mbarriers (8 B each)
 
 enum Bar : int {
-    kBarQ = 0,       // Q landed (TMA transaction bytes)
-    kBarKvFull = 1,  // bf16 tile written (16 warp arrivals after a proxy fence)
-    kBarSFull = 2,   // S^T complete (MMA commit)
-    kBarPFull = 3,   // P^T written (16 warp arrivals after a proxy fence)
-    kBarPvDone = 4,  // PV complete (MMA commit): tile buffers and O^T free
-    kBarDrain = 5,   // final commit before tensor memory is released
-    kBarSpare = 6,   // test hook target
-    kBarRecv = 7,    // cluster merge: partials received from the other CTAs (bulk-copy bytes)
+    kBarQ = 0,        // Q landed (TMA transaction bytes)
+    kBarKvFull = 1,   // + c (c = 0..3): K-block pair c of the tile written (8 producer-warp arrivals)
+    kBarKvFree = 5,   // + c: PV chunk c of the tile done (MMA commit): pair c may be overwritten
+    kBarSFull = 9,    // + s (s = 0..1): S^T buffer s complete (MMA commit)
+    kBarPFull = 11,   // P^T written (8 softmax-warp arrivals)
+    kBarDrain = 12,   // final commit before tensor memory is released
+    kBarSpare = 13,   // test hook target
+    kBarXch = 14,     // cluster merge: the other CTAs' rows and chunks landed (bulk-copy bytes)
+    kNumBars = 15,
 };
+constexpr int kSmemTmemSlot = kSmemBars + kNumBars * 8;
+constexpr int kSmemAbort = kSmemTmemSlot + 4;
+constexpr int kSmemBytes = kSmemAbort + 4;
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory limit");
+static_assert(kSmemBars % 8 == 0, "mbarriers need 8-byte alignment");
 
-constexpr uint32_t kTmemCols = 512;  // O^T [0,256), S^T [256,320), per-lane running sums [320,384)
+// Tensor memory: O^T [0,256) (4 chunks of 128 dims x 64 heads), S^T buffers at 256 and 320.
+constexpr int kMlBytes = 128 * 4;  // one (m, l) row of the cluster merge
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;
-constexpr uint32_t kTmemL = 320;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, true, true);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(s - m) stays below 256 without a rescale
@@ -99,17 +112,18 @@ struct DecodeParams {
     int tiles_per_split;
     float scale_log2;  // sm_scale * log2(e)
     uint32_t debug_flags;
-    int cluster_merge;  // 1: the nsplit CTAs of a request form a cluster and merge through DSMEM
+    int cluster_merge;  // 1: the nsplit CTAs of a request form a cluster and merge in the kernel
 };
 
-// Reduces 16 per-thread values across the 32 lanes of a warp, value i with value i
-// of every other lane.  Afterwards lanes 2j and 2j+1 both hold the result for entry
-// j.  Each round halves the live entries: a lane keeps the half selected by its
-// lane bit and sends the other half to its partner; the last round combines pairs.
-template <bool kMax>
-__device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16], int lane) {
+// Reduces N (16 or 32) per-thread values across the 32 lanes of a warp, value i with
+// value i of every other lane.  Each round halves the live entries: a lane keeps the
+// half selected by its lane bit and sends the other half to its partner.  With N = 32
+// lane j ends with entry j; with N = 16 lanes 2j and 2j+1 end with entry j.
+template <bool kMax, int N>
+__device__ __forceinline__ float warp_transpose_reduce(float (&v)[N], int lane) {
+    static_assert(N == 16 || N == 32, "16 or 32 entries");
 #pragma unroll
-    for (int w = 8, off = 16; off >= 2; w >>= 1, off >>= 1) {
+    for (int w = N / 2, off = 16; w >= 1; w >>= 1, off >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < w; ++i) {
@@ -119,8 +133,11 @@ __device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16], int lan
             v[i] = kMax ? fmaxf(keep, got) : keep + got;
         }
     }
-    const float got = __shfl_xor_sync(0xffffffffu, v[0], 1);
-    return kMax ? fmaxf(v[0], got) : v[0] + got;
+    if constexpr (N == 16) {
+        const float got = __shfl_xor_sync(0xffffffffu, v[0], 1);
+        return kMax ? fmaxf(v[0], got) : v[0] + got;
+    }
+    return v[0];
 }
 
 // Bounded wait on an mbarrier phase.  Gives up when another thread has aborted the
@@ -152,19 +169,19 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
 }
 
 // ------------------------------------------------------------------ gather + dequant
-// The 128 x 36 sixteen-byte chunks of a tile are dealt out in four groups, one per
-// K-block pair c (dims [128c, 128c+128)):
-//   pairs 0..2: 128 tokens x 8 nope chunks (16 dims)          -> 2 items per thread
-//   pair 3:     128 tokens x (4 nope + 8 rope chunks)          -> 3 items per thread
+// The 128 x 36 sixteen-byte chunks of a tile are dealt out to the 256 producer threads
+// in four groups, one per K-block pair c (dims [128c, 128c+128)):
+//   pairs 0..2: 128 tokens x 8 nope chunks (16 dims)          -> 4 items per thread
+//   pair 3:     128 tokens x (4 nope + 8 rope chunks)          -> 6 items per thread
 // Consecutive threads take consecutive chunks of a token row (coalesced loads).
 template <int C>
 struct PairShape {
-    static constexpr int kItems = (C < 3) ? 2 : 3;
+    static constexpr int kItems = (C < 3) ? 4 : 6;
 };
 
 template <int C>
 __device__ __forceinline__ void pair_item(int t, int u, int &r, int &chunk, int &kb, int &oc, bool &nope) {
-    const int j = t + kThreads * u;
+    const int j = t + kProducerThreads * u;
     if constexpr (C < 3) {
         r = j >> 3;
         const int k = j & 7;
@@ -189,43 +206,59 @@ __device__ __forceinline__ void pair_item(int t, int u, int &r, int &chunk, int 
     }
 }
 
-// The FP8 bytes (and the scale byte) of one tile, held in registers between the
-// load and the dequantisation.
+// The FP8 bytes of one tile and their scales, held in registers between the load and
+// the dequantisation.  In pairs 0..2 a producer thread always takes chunk (pt & 7) of the
+// four tokens (pt >> 3) + 32u, so it loads each of those tokens' 8-byte scale row once
+// (srow[u]); in pair 3 it loads the one scale byte an item needs.
 struct TileRegs {
-    uint4 raw0[2], raw1[2], raw2[2], raw3[3];
-    uint32_t sc0[2], sc1[2], sc2[2], sc3[3];
+    uint4 raw0[4], raw1[4], raw2[4], raw3[6];
+    uint2 srow[4];
+    uint32_t sc3[6];
 };
 
-template <int C>
-__device__ __forceinline__ void load_pair(int t, const int *codes, const uint8_t *cache,
-                                          uint4 (&raw)[PairShape<C>::kItems], uint32_t (&sc)[PairShape<C>::kItems]) {
+__device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t *cache, TileRegs &tr) {
 #pragma unroll
-    for (int u = 0; u < PairShape<C>::kItems; ++u) {
+    for (int u = 0; u < 4; ++u) {
+        const int r = (t >> 3) + 32 * u;
+        const int chunk = t & 7;
+        const int code = codes[r];
+        tr.raw0[u] = tr.raw1[u] = tr.raw2[u] = make_uint4(0u, 0u, 0u, 0u);
+        tr.srow[u] = make_uint2(0u, 0u);
+        if (code >= 0) {
+            const uint8_t *row = token_row(cache, code);
+            tr.raw0[u] = ld_stream_v4(row + chunk * 16);
+            tr.raw1[u] = ld_stream_v4(row + (8 + chunk) * 16);
+            tr.raw2[u] = ld_stream_v4(row + (16 + chunk) * 16);
+            tr.srow[u] = ld_stream_v2(token_scales(cache, code));
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 6; ++u) {
         int r, chunk, kb, oc;
         bool nope;
-        pair_item<C>(t, u, r, chunk, kb, oc, nope);
+        pair_item<3>(t, u, r, chunk, kb, oc, nope);
         const int code = codes[r];
-        raw[u] = make_uint4(0u, 0u, 0u, 0u);
-        sc[u] = 0u;
+        tr.raw3[u] = make_uint4(0u, 0u, 0u, 0u);
+        tr.sc3[u] = 0u;
         if (code >= 0) {
-            raw[u] = ld_stream_v4(token_row(cache, code) + chunk * 16);
-            if (nope) sc[u] = ld_stream_u8(token_scales(cache, code) + (chunk >> 2));
+            tr.raw3[u] = ld_stream_v4(token_row(cache, code) + chunk * 16);
+            if (nope) tr.sc3[u] = ld_stream_u8(token_scales(cache, code) + (chunk >> 2));
         }
     }
 }
 
-__device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t *cache, TileRegs &tr) {
-    load_pair<0>(t, codes, cache, tr.raw0, tr.sc0);
-    load_pair<1>(t, codes, cache, tr.raw1, tr.sc1);
-    load_pair<2>(t, codes, cache, tr.raw2, tr.sc2);
-    load_pair<3>(t, codes, cache, tr.raw3, tr.sc3);
+// Scale byte of item u of pair C (C < 3): byte 2C + ((t & 7) >> 2) of the token's scale row.
+template <int C>
+__device__ __forceinline__ uint32_t pair_scale(const TileRegs &tr, int t, int u) {
+    const int byte = 2 * C + ((t & 7) >> 2);
+    const uint32_t w = (byte < 4) ? tr.srow[u].x : tr.srow[u].y;
+    return (w >> (8 * (byte & 3))) & 0xFFu;
 }
 
 // Dequantises this thread's items of pair C into the swizzled bf16 tile (plain shared
 // stores; `kv` is the tile's shared-window address).
 template <int C>
-__device__ __forceinline__ void store_pair(int t, uint32_t kv, const uint4 (&raw)[PairShape<C>::kItems],
-                                           const uint32_t (&sc)[PairShape<C>::kItems]) {
+__device__ __forceinline__ void store_pair(int t, uint32_t kv, const TileRegs &tr) {
 #pragma unroll
     for (int u = 0; u < PairShape<C>::kItems; ++u) {
         int r, chunk, kb, oc;
@@ -233,9 +266,24 @@ __device__ __forceinline__ void store_pair(int t, uint32_t kv, const uint4 (&raw
         pair_item<C>(t, u, r, chunk, kb, oc, nope);
         const uint32_t row = kv + kb * (kTile * 128) + r * 128;
         const int sw = r & 7;
+        uint4 raw;
+        uint32_t sc;
+        if constexpr (C == 0) {
+            raw = tr.raw0[u];
+            sc = pair_scale<C>(tr, t, u);
+        } else if constexpr (C == 1) {
+            raw = tr.raw1[u];
+            sc = pair_scale<C>(tr, t, u);
+        } else if constexpr (C == 2) {
+            raw = tr.raw2[u];
+            sc = pair_scale<C>(tr, t, u);
+        } else {
+            raw = tr.raw3[u];
+            sc = tr.sc3[u];
+        }
         if (nope) {
             uint4 lo, hi;
-            dequant16(raw[u], sc[u], lo, hi);
+            dequant16(raw, sc, lo, hi);
             // odd K-blocks store their high half first so the 8 lanes of a store phase hit 8 bank groups
             if ((kb & 1) == 0) {
                 sts_v4(row + ((oc ^ sw) << 4), lo);
@@ -245,169 +293,252 @@ __device__ __forceinline__ void store_pair(int t, uint32_t kv, const uint4 (&raw
                 sts_v4(row + ((oc ^ sw) << 4), lo);
             }
         } else {
-            sts_v4(row + ((oc ^ sw) << 4), raw[u]);
+            sts_v4(row + ((oc ^ sw) << 4), raw);
         }
     }
 }
 
+// Producer step for pair C of a tile: wait until the PV of the previous tile has
+// released the pair, dequantise into it, publish it to the tensor core.
+template <int C>
+__device__ __forceinline__ bool produce_pair(int i, int pt, int lane, uint32_t kv_s, uint64_t *bars,
+                                             volatile int *abort_flag, const DecodeParams &p, const TileRegs &tr) {
+    if (i > 0 && !warp_wait_phase(&bars[kBarKvFree + C], (i - 1) & 1, abort_flag, p, lane)) return false;
+    store_pair<C>(pt, kv_s, tr);
+    fence_proxy_async_smem();  // this thread's stores -> visible to the tensor core
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarKvFull + C]);
+    return true;
+}
+
 // ------------------------------------------------------------------ split merge in a cluster
-// The nsplit CTAs of one request form a thread-block cluster.  After the last PV,
-// CTA s holds un-normalised O^T_s (tensor memory), its per-head running max m_s (log2
-// units) and sum l_s.  With L = log2 sum_s 2^(m_s) l_s, the merged output is
-// O = sum_s 2^(m_s - L) O^T_s and LSE = L ln 2 (the split-K log-sum-exp merge).
-// Output dims are dealt out by 128-dim chunk: chunk mc belongs to CTA mc % nsplit.
-// Once every CTA's MMAs are done (its Q, KV and P buffers are dead), each CTA stages
-// its (m_s, l_s) row and the O^T_s chunks it does not own in its own shared memory
-// and sends them with bulk shared-to-shared copies into the owners' receive areas,
-// where they are counted in bytes on kBarRecv.  Receive area of a CTA: blocks
-// [owned chunk lci][sender slot] from offset 0, the (m, l) rows at kSmemMl; its send
-// staging follows its receive blocks.
-constexpr int kRecvRow = 272;               // 64 heads x fp32 + 16 B pad: conflict-free row stores
-constexpr int kRecvBlock = 128 * kRecvRow;  // one 128-dim chunk of O^T
-constexpr int kMlRow = 512;                 // m[64] | l[64], f32
+// The nsplit (2..4) CTAs of one request form a thread-block cluster, which makes them
+// co-resident.  After the last PV, CTA s holds un-normalised O^T_s (tensor memory), its
+// per-head running max m_s (log2 units) and sum l_s.  With L = log2 sum_s 2^(m_s) l_s,
+// the merged output is O = sum_s 2^(m_s - L) O^T_s and LSE = L ln 2 (the split-K
+// log-sum-exp merge).  Output dims are dealt out by 128-dim chunk: chunk mc belongs to
+// CTA mc % nsplit.  Each CTA publishes its (m_s, l_s) row and the O^T_s chunks it does
+// not own to the workspace (coalesced stores that stay in L2); after one cluster barrier
+// (release / acquire) each owner pulls what it needs into its own shared memory with
+// bulk copies counted on one mbarrier (a single L2 round trip), then merges.
+// Distributed shared memory is not used for the exchange: its per-SM bandwidth is a
+// fraction of what L2 gives one SM.
+//   ml   [B][nsplit][m(64) | l(64)] f32
+//   xch  [B][4 chunks][nsplit - 1 sender slots][64 heads][128 dims] f32 (a warp's
+//        32 consecutive dims are one 128-byte line); the sender slot of CTA s in
+//        chunk mc is s, minus one when s is above the owner.
+// Shared memory (the operand buffers are dead by then): the rows at the Q buffer
+// [nsplit][128] f32, the received chunks at the KV buffer [owned chunk][sender slot]
+// [64][128] f32.
+// Called by every thread of the CTA (the cluster barrier needs them all); the softmax
+// warps (quadrant q, head half hh) do the work.
+constexpr int kXchBlock = kHeads * 128 * 4;  // one 128-dim chunk of O^T, bytes
 
-__host__ __device__ constexpr int owned_chunks(int me, int ns) { return (4 - me + ns - 1) / ns; }
-static_assert(4 * kRecvBlock + 2 * kRecvBlock <= kSmemMl, "receive + send areas overlap the (m, l) rows");
-static_assert(3 * kRecvBlock + 3 * kRecvBlock <= kSmemMl, "receive + send areas overlap the (m, l) rows");
-
-__device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool ok, int n, int tid, int q, int g,
-                                              int lane, uint32_t tmem, uint32_t lane_base, uint8_t *smem,
-                                              uint64_t *bar_recv, const float *head_m, const float *l_head,
-                                              float *weights) {
+__device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool ok, int n, int tid, int warp,
+                                              int lane, uint32_t tmem, uint8_t *smem, uint64_t *bar_xch,
+                                              const float *head_m, const float *l_head, float *weights) {
     const int ns = p.nsplit;
     const int me = static_cast<int>(cluster_ctarank());
-    const int n_own = owned_chunks(me, ns);
-    const uint32_t base = smem_addr(smem);
-    const uint32_t send = base + n_own * (ns - 1) * kRecvBlock;
-    float *ml = reinterpret_cast<float *>(smem + kSmemMl);  // [s][m(64) | l(64)]
-    const int d = 32 * q + lane;                            // row of O^T within a chunk
+    const int n_own = (4 - me + ns - 1) / ns;  // chunks me, me + ns, ... below 4
+    const bool worker = warp < kSoftmaxWarps;
+    const int q = warp & 3, hh = (warp >> 2) & 1;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const int d = 32 * q + lane;  // row of O^T within a chunk
     const bool live = ok && n > 0;
+    float *ml = p.part_lse + static_cast<size_t>(b) * ns * 128;
+    float *xch = p.part_o + static_cast<size_t>(b) * 4 * (ns - 1) * (kHeads * 128);
+    float *ml_s = reinterpret_cast<float *>(smem + kSmemQ);
+    const float *recv = reinterpret_cast<const float *>(smem + kSmemKV);
 
-    // barrier 1: every CTA's MMAs are done, so its operand buffers may be overwritten
-    cluster_sync();
     if (tid < kHeads) {
-        ml[me * 128 + tid] = live ? head_m[tid] : -INFINITY;
-        ml[me * 128 + 64 + tid] = live ? l_head[tid] : 0.0f;
+        const float mv = live ? head_m[tid] : -INFINITY;
+        const float lv = live ? l_head[tid] : 0.0f;
+        ml[me * 128 + tid] = mv;
+        ml[me * 128 + 64 + tid] = lv;
+        ml_s[me * 128 + tid] = mv;
+        ml_s[me * 128 + 64 + tid] = lv;
     }
-    {
-        int js = 0;
+    if (worker) {
 #pragma unroll 1
-        for (int mc = 0; mc < 4; ++mc) {
-            if (mc % ns == me) continue;
-            float o[16];
-            if (live) {
-                tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, o);
-                tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int h = 0; h < 16; ++h) o[h] = 0.0f;
-            }
-            const uint32_t row = send + js * kRecvBlock + d * kRecvRow + 64 * g;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) sts_v4f(row + 16 * j, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-            ++js;
-        }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid < ns && tid != me) {
-        const int peer = tid;
-        const uint32_t bar_c = map_to_rank(bar_recv, peer);
-        bulk_copy_to_cluster(map_to_rank(ml + me * 128, peer), smem_addr(ml + me * 128), kMlRow, bar_c);
-        int js = 0;
         for (int mc = 0; mc < 4; ++mc) {
             const int owner = mc % ns;
             if (owner == me) continue;
-            if (owner == peer) {
-                const int slot = (me < peer) ? me : me - 1;
-                const int blk = (mc / ns) * (ns - 1) + slot;
-                bulk_copy_to_cluster(map_to_rank(smem + blk * kRecvBlock, peer), send + js * kRecvBlock, kRecvBlock,
-                                     bar_c);
+            float o[32];
+            if (live) {
+                tmem_ld32(tmem + lane_base + 64 * mc + 32 * hh, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int h = 0; h < 32; ++h) o[h] = 0.0f;
             }
-            ++js;
+            const int slot = (me < owner) ? me : me - 1;
+            float *dst = xch + ((mc * (ns - 1) + slot) * kHeads + 32 * hh) * 128 + d;
+#pragma unroll
+            for (int h = 0; h < 32; ++h) __stcg(dst + h * 128, o[h]);
         }
     }
-    // the other CTAs' rows and chunks have landed (bounded wait; the copies are in flight
-    // whatever happened elsewhere, so the abort flag does not cut it short)
+    fence_proxy_async_all();  // the peers read these rows and chunks with bulk copies
+    // every CTA's row and chunks are written before any owner fetches them
+    cluster_sync();
     int got = 1;
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_recv, (ns - 1) * (kMlRow + n_own * kRecvBlock));
-        got = mbar_wait(bar_recv, 0, p.timeout_ns) ? 1 : 0;
+        fence_proxy_async_all();
+        mbar_arrive_expect_tx(bar_xch, (ns - 1) * (kMlBytes + n_own * kXchBlock));
+        for (int s = 0; s < ns; ++s) {
+            if (s == me) continue;
+            bulk_load(ml_s + s * 128, ml + s * 128, kMlBytes, bar_xch);
+            const int slot = (s < me) ? s : s - 1;
+            for (int lci = 0; lci < n_own; ++lci) {
+                const int mc = me + lci * ns;
+                bulk_load(smem + kSmemKV + (lci * (ns - 1) + slot) * kXchBlock,
+                          xch + (mc * (ns - 1) + slot) * (kHeads * 128), kXchBlock, bar_xch);
+            }
+        }
+        got = mbar_wait(bar_xch, 0, p.timeout_ns) ? 1 : 0;
         if (!got) atomicOr(p.err, SMLA_FLAG_TIMEOUT);
     }
     got = __syncthreads_and(got);
-    if (got) (void)mbar_try_wait(bar_recv, 0);  // every thread observes the completed phase
-    const bool write = got && ok;
+    if (got) (void)mbar_try_wait(bar_xch, 0);  // every thread observes the completed phase
+    const bool write = ok && got;
     if (tid < kHeads) {
         float mx = -INFINITY;
         for (int s = 0; s < ns; ++s)
-            if (ml[s * 128 + 64 + tid] > 0.0f) mx = fmaxf(mx, ml[s * 128 + tid]);
+            if (ml_s[s * 128 + 64 + tid] > 0.0f) mx = fmaxf(mx, ml_s[s * 128 + tid]);
         float sum = 0.0f;
         for (int s = 0; s < ns; ++s) {
-            const float l = ml[s * 128 + 64 + tid];
-            if (l > 0.0f) sum += exp2f(ml[s * 128 + tid] - mx) * l;
+            const float lv = ml_s[s * 128 + 64 + tid];
+            if (lv > 0.0f) sum += exp2f(ml_s[s * 128 + tid] - mx) * lv;
         }
         const float L = (sum > 0.0f) ? mx + log2f(sum) : -INFINITY;
-        for (int s = 0; s < ns; ++s)
-            weights[s * kHeads + tid] = (sum > 0.0f && ml[s * 128 + 64 + tid] > 0.0f) ? exp2f(ml[s * 128 + tid] - L)
-                                                                                      : 0.0f;
+        for (int s = 0; s < ns; ++s) {
+            const float lv = ml_s[s * 128 + 64 + tid];
+            weights[s * kHeads + tid] = (sum > 0.0f && lv > 0.0f) ? exp2f(ml_s[s * 128 + tid] - L) : 0.0f;
+        }
         if (me == 0 && write)
             p.lse[static_cast<size_t>(b) * kHeads + tid] = (sum > 0.0f) ? L * 0.69314718055994531f : -INFINITY;
     }
     __syncthreads();
-    if (write) {
+    if (!write || !worker) return;
 #pragma unroll 1
-        for (int mc = me; mc < 4; mc += ns) {
-            const int lci = mc / ns;
-            float acc[16];
-            if (live) {
-                tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, acc);
-                tmem_wait_ld();
-            }
-#pragma unroll
-            for (int h = 0; h < 16; ++h) {
-                const float w = weights[me * kHeads + 16 * g + h];
-                acc[h] = (live && w != 0.0f) ? acc[h] * w : 0.0f;
-            }
-            for (int s = 0; s < ns; ++s) {
-                if (s == me) continue;
-                const int slot = (s < me) ? s : s - 1;
-                const float4 *src = reinterpret_cast<const float4 *>(smem + (lci * (ns - 1) + slot) * kRecvBlock +
-                                                                     d * kRecvRow + 64 * g);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 v = src[j];
-                    const float *w = weights + s * kHeads + 16 * g + 4 * j;
-                    if (w[0] != 0.0f) acc[4 * j] += v.x * w[0];
-                    if (w[1] != 0.0f) acc[4 * j + 1] += v.y * w[1];
-                    if (w[2] != 0.0f) acc[4 * j + 2] += v.z * w[2];
-                    if (w[3] != 0.0f) acc[4 * j + 3] += v.w * w[3];
-                }
-            }
-            float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * g) * kDim + 128 * mc + d;
-#pragma unroll
-            for (int h = 0; h < 16; ++h) dst[h * kDim] = acc[h];
+    for (int lci = 0; lci < n_own; ++lci) {
+        const int mc = me + lci * ns;
+        float acc[32];
+        if (live) {
+            tmem_ld32(tmem + lane_base + 64 * mc + 32 * hh, acc);
+            tmem_wait_ld();
         }
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+            const float w = weights[me * kHeads + 32 * hh + h];
+            acc[h] = (live && w != 0.0f) ? acc[h] * w : 0.0f;
+        }
+        for (int s = 0; s < ns; ++s) {
+            if (s == me) continue;
+            const int slot = (s < me) ? s : s - 1;
+            const float *src = recv + ((lci * (ns - 1) + slot) * kHeads + 32 * hh) * 128 + d;
+#pragma unroll
+            for (int h = 0; h < 32; ++h) {
+                const float w = weights[s * kHeads + 32 * hh + h];
+                if (w != 0.0f) acc[h] += src[h * 128] * w;
+            }
+        }
+        float *dst = p.out + (static_cast<size_t>(b) * kHeads + 32 * hh) * kDim + 128 * mc + d;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) dst[h * kDim] = acc[h];
     }
-    // barrier 2: no CTA leaves while a bulk copy may still be reading its staging area
-    cluster_sync();
 }
 
+// ------------------------------------------------------------------ MMA issue
+// The tensor-core side of the pipeline, run by one thread.  Every wait is bounded; a
+// failed wait leaves `ok` false and issues nothing more.
+struct MmaIssuer {
+    uint64_t dQK_a, dQK_b, dPV_a, dPV_bh, dPV_bl;
+    uint32_t tmem;
+    const DecodeParams &p;
+    uint64_t *bars;
+    volatile int *abort_flag;
+    bool ok = true;
+    bool spare_used = false;
+
+    __device__ MmaIssuer(uint8_t *smem, uint32_t tmem_, const DecodeParams &p_, uint64_t *bars_,
+                         volatile int *abort_)
+        : tmem(tmem_), p(p_), bars(bars_), abort_flag(abort_) {
+        dQK_a = sw128_desc(smem_addr(smem + kSmemKV), 16, 1024);
+        dQK_b = sw128_desc(smem_addr(smem + kSmemQ), 16, 1024);
+        dPV_a = sw128_desc(smem_addr(smem + kSmemKV), kTile * 128, 1024);
+        dPV_bh = sw128_desc(smem_addr(smem + kSmemPhi), 8192, 1024);
+        dPV_bl = sw128_desc(smem_addr(smem + kSmemPlo), 8192, 1024);
+    }
+
+    // S^T[tile i] = K.Q^T into buffer i&1, one K-block pair as soon as it is published.
+    __device__ void qk(int i) {
+        if (!ok) return;
+        const uint32_t s_col = tmem + kTmemS + 64 * (i & 1);
+#pragma unroll
+        for (int cp = 0; cp < 4; ++cp) {
+            ok = ok && (i > 0 || cp > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
+                 wait_phase(&bars[kBarKvFull + cp], i & 1, abort_flag, p);
+            if (!ok) return;
+            tc_fence_after_sync();
+#pragma unroll
+            for (int kb = 2 * cp; kb < 2 * cp + 2; ++kb)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(s_col, dQK_a + (kb * (kTile * 128) + kk * 32) / 16, dQK_b + (kb * 8192 + kk * 32) / 16,
+                                kIdescQK, (kb | kk) != 0);
+        }
+        const bool hook = (i == 0) && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
+        mma_commit(hook ? &bars[kBarSpare] : &bars[kBarSFull + (i & 1)]);
+        spare_used = spare_used || hook;
+    }
+
+    // O^T += V^T.P_hi^T + V^T.P_lo^T of tile i once every softmax warp has written P^T;
+    // each 128-dim chunk is committed to the producers as it completes.
+    __device__ bool pv(int i) {
+        if (!ok) return false;
+        ok = wait_phase(&bars[kBarPFull], i & 1, abort_flag, p);
+        if (!ok) return false;
+        tc_fence_after_sync();
+        const uint32_t acc0 = (i > 0) ? 1u : 0u;
+#pragma unroll
+        for (int mc = 0; mc < 4; ++mc) {
+            const uint64_t a0 = dPV_a + static_cast<uint64_t>(mc * 2 * (kTile * 128 / 16));
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bh + ks * (2048 / 16), kIdescPV,
+                            ks > 0 ? 1u : acc0);
+                mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bl + ks * (2048 / 16), kIdescPV, 1u);
+            }
+            mma_commit(&bars[kBarKvFree + mc]);
+        }
+        return true;
+    }
+
+    __device__ void drain() {
+        if (spare_used) (void)mbar_wait(&bars[kBarSpare], 0, p.timeout_ns);
+        mma_commit(&bars[kBarDrain]);
+        (void)mbar_wait(&bars[kBarDrain], 0, p.timeout_ns);
+    }
+};
+
 // ------------------------------------------------------------------ the decode kernel
-// One CTA per (topk split, request), 16 warps, one 128-slot tile at a time:
-//   1. every thread dequantises its 9 prefetched chunks of the tile into the bf16
-//      tile (plain shared stores, a proxy fence, one mbarrier arrival per warp);
-//   2. every thread issues the loads of the next tile (they stay in flight through
-//      the MMA and softmax phases), and threads 0..127 run the index translation of
-//      the tile after next, spread over the phases so its latency is hidden;
-//   3. thread 0 issues S^T = K.Q^T (32 tcgen05.mma, M=128 tokens, N=64 heads);
-//   4. softmax on all 16 warps: warp w reads TMEM lanes 32(w%4).. (tokens) and
-//      columns 16(w/4).. (heads); p = 2^(s*c - m) against the running max m, which
-//      is raised (with a rescale of O^T and of the per-lane running sums) only when a
-//      score exceeds it by more than 2^8; P^T is written as bf16 hi + lo terms;
-//   5. thread 0 issues O^T += V^T.P_hi^T + V^T.P_lo^T (64 tcgen05.mma).
-// The epilogue reduces the per-lane sums and writes O/l and LSE, merging the splits of
-// a request inside its thread-block cluster when there are several.
+// One CTA per (topk split, request), one 128-slot tile at a time, three warp roles
+// that hand work to each other through mbarriers:
+//   producers (8 warps): translate the slots of tile i+2 through the block table,
+//     keep the FP8 rows of tile i+1 in flight in registers, and dequantise tile i
+//     into the bf16 tile one K-block pair at a time, each pair as soon as the PV of
+//     tile i-1 has released it (so dequantisation overlaps the previous PV);
+//   MMA issue (lane 0 of softmax warp 0, between its softmax steps): once P^T of tile
+//     i is written, O^T += V^T.P_hi^T + V^T.P_lo^T (64 MMAs), committing each 128-dim
+//     chunk to the producers; then S^T = K.Q^T of tile i+1 (M=128 tokens, N=64
+//     heads) pair by pair as the producers publish them, into the other of two S^T
+//     buffers in tensor memory;
+//   softmax (8 warps; warp w reads TMEM lanes 32(w%4).. = tokens, columns for heads
+//     32(w/4)..): p = 2^(s*c - m) against the running max m, which is raised (with a
+//     rescale of O^T and of the per-thread sums) only when a score exceeds it by more
+//     than 2^8; P^T is written as bf16 hi + lo terms.
+// The epilogue reduces the per-thread sums and writes O/l and LSE, merging the splits of
+// a request inside its thread-block cluster when there are 2..4 of them.
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_q) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -423,9 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     uint8_t *sQ = smem + kSmemQ;
     uint8_t *sKV = smem + kSmemKV;
-    uint8_t *sPhi = smem + kSmemPhi;
-    uint8_t *sPlo = smem + kSmemPlo;
     int *codes = reinterpret_cast<int *>(smem + kSmemCodes);
+    uint32_t *mask = reinterpret_cast<uint32_t *>(smem + kSmemMask);
     float *head_m = reinterpret_cast<float *>(smem + kSmemHeadM);
     float *head_alpha = reinterpret_cast<float *>(smem + kSmemHeadAlpha);
     float *red = reinterpret_cast<float *>(smem + kSmemRed);
@@ -440,248 +570,205 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t *bt_row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
     const int32_t *idx_row = p.topk_idx + static_cast<size_t>(b) * p.topk;
 
+    // ---- setup
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
-    }
-    if (tid == 32) {
-        mbar_init(&bars[kBarQ], 1);
-        mbar_init(&bars[kBarKvFull], 16);
-        mbar_init(&bars[kBarSFull], 1);
-        mbar_init(&bars[kBarPFull], 16);
-        mbar_init(&bars[kBarPvDone], 1);
-        mbar_init(&bars[kBarDrain], 1);
-        mbar_init(&bars[kBarSpare], 1);
-        mbar_init(&bars[kBarRecv], 1);
-        fence_barrier_init();
-        *abort_flag = 0;
-        mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
+        if (lane == 0) {
+            mbar_init(&bars[kBarQ], 1);
+            for (int c = 0; c < 4; ++c) {
+                mbar_init(&bars[kBarKvFull + c], kProducerWarps);
+                mbar_init(&bars[kBarKvFree + c], 1);
+            }
+            mbar_init(&bars[kBarSFull], 1);
+            mbar_init(&bars[kBarSFull + 1], 1);
+            mbar_init(&bars[kBarPFull], kSoftmaxWarps);
+            mbar_init(&bars[kBarDrain], 1);
+            mbar_init(&bars[kBarSpare], 1);
+            mbar_init(&bars[kBarXch], 1);
+            fence_barrier_init();
+            *abort_flag = 0;
+            mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
 #pragma unroll
-        for (int kb = 0; kb < 8; ++kb) tma_load_2d(sQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
-    }
-    if (tid < kHeads) head_m[tid] = -INFINITY;
-    // index translation of tiles 0 and 1 (threads 0..255: tile tid/128, slot tid%128)
-    if (tid < 2 * kTile) {
-        const int ti = tid >> 7;
-        const int slot = (t_begin + ti) * kTile + (tid & (kTile - 1));
+            for (int kb = 0; kb < 8; ++kb) tma_load_2d(sQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
+        }
+    } else if (warp >= kSoftmaxWarps) {
+        // index translation of tiles 0 and 1 (producer thread pt: tile pt/128, slot pt%128)
+        const int pt = tid - kSoftmaxThreads;
+        const int ti = pt >> 7;
+        const int slot = (t_begin + ti) * kTile + (pt & (kTile - 1));
         int code = -1;
         if (ti < n && slot < p.topk)
             code = translate_slot(bt_row, p.max_blocks, seq_len, p.num_pages, __ldg(idx_row + slot), p.err);
-        codes[tid] = code;
+        codes[pt] = code;
+        const uint32_t bits = __ballot_sync(0xffffffffu, code >= 0);
+        if (lane == 0) mask[ti * 4 + ((pt >> 5) & 3)] = bits;
     }
+    if (tid < kHeads) head_m[tid] = -INFINITY;
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t kv_s = smem_addr(sKV);
-    const uint32_t phi_s = smem_addr(sPhi);
-    const uint32_t plo_s = smem_addr(sPlo);
-
-    // thread roles inside the softmax / epilogue: TMEM lane quadrant q, head group g
-    const int q = warp & 3;
-    const int g = warp >> 2;
-    const int r = 32 * q + lane;  // token lane of S^T, output-dim lane of O^T
-    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const float c = p.scale_log2;
 
-    // MMA descriptors of the operand bases; every MMA adds a compile-time offset (bytes >> 4)
-    const uint64_t dQK_a = sw128_desc(smem_addr(sKV), 16, 1024);
-    const uint64_t dQK_b = sw128_desc(smem_addr(sQ), 16, 1024);
-    const uint64_t dPV_a = sw128_desc(smem_addr(sKV), kTile * 128, 1024);
-    const uint64_t dPV_bh = sw128_desc(smem_addr(sPhi), 8192, 1024);
-    const uint64_t dPV_bl = sw128_desc(smem_addr(sPlo), 8192, 1024);
-
-    TileRegs tr;
-    if (n > 0) load_tile(tid, codes, p.cache, tr);
-    bool failed = false, spare_used = false;
-    int idx_next = -1, page_next = -1;
-
-    for (int i = 0; i < n; ++i) {
-        const int buf = i & 1;
-        const bool valid = codes[buf * kTile + r] >= 0;
-        // ---- 1. dequantise the tile
-        store_pair<0>(tid, kv_s, tr.raw0, tr.sc0);
-        store_pair<1>(tid, kv_s, tr.raw1, tr.sc1);
-        store_pair<2>(tid, kv_s, tr.raw2, tr.sc2);
-        store_pair<3>(tid, kv_s, tr.raw3, tr.sc3);
-        fence_proxy_async_smem();  // this thread's tile stores -> visible to the tensor core
+    if (warp < kSoftmaxWarps) {
+        // ================================================================ softmax (+ MMA issue)
+        const int q = warp & 3;
+        const int hh = warp >> 2;
+        const int r = 32 * q + lane;  // token lane of S^T
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        const uint32_t phi_s = smem_addr(smem + kSmemPhi);
+        const uint32_t plo_s = smem_addr(smem + kSmemPlo);
+        const bool issuer = (tid == 0);
+        MmaIssuer mma(smem, tmem, p, bars, abort_flag);
+        if (issuer && n > 0) mma.qk(0);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarKvFull]);
-        // ---- 2. prefetch the next tile, start translating the tile after it
-        if (i + 1 < n) load_tile(tid, codes + (buf ^ 1) * kTile, p.cache, tr);
-        const int slot2 = (t_begin + i + 2) * kTile + tid;
-        if (tid < kTile && i + 2 < n && slot2 < p.topk) idx_next = __ldg(idx_row + slot2);
-        // ---- 3. S^T = K.Q^T
-        if (tid == 0) {
-            bool ok = (i > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
-                      wait_phase(&bars[kBarKvFull], i & 1, abort_flag, p);
-            if (ok) {
-                tc_fence_after_sync();
+        float l[32];
 #pragma unroll
-                for (int kb = 0; kb < 8; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + kTmemS, dQK_a + (kb * (kTile * 128) + kk * 32) / 16,
-                                    dQK_b + (kb * 8192 + kk * 32) / 16, kIdescQK, (kb | kk) != 0);
-                const bool hook = (i == 0) && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
-                mma_commit(hook ? &bars[kBarSpare] : &bars[kBarSFull]);
-                spare_used = hook;
+        for (int h = 0; h < 32; ++h) l[h] = 0.0f;
+        bool failed = false;
+        for (int i = 0; i < n; ++i) {
+            const int sb = i & 1;
+            const uint32_t s_cols = tmem + lane_base + kTmemS + 64 * sb + 32 * hh;
+            const bool ok = warp_wait_phase(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag, p, lane);
+            if (barrier_or(kBarIdSoftmax, kSoftmaxThreads, !ok)) {
+                failed = true;
+                break;
             }
-        }
-        bool ok = warp_wait_phase(&bars[kBarSFull], i & 1, abort_flag, p, lane);
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        tc_fence_after_sync();
-        if (tid < kTile && i + 2 < n && idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks)
-            page_next = __ldg(bt_row + (idx_next >> 8));
-        // ---- 4. online softmax over 16 warps
-        float x[16];
-        tmem_ld16(tmem + lane_base + kTmemS + 16 * g, x);
-        tmem_wait_ld();
-        bool over = false;
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-            x[h] = valid ? fmaf(x[h], c, -head_m[16 * g + h]) : -INFINITY;
-            over |= x[h] > kRescaleThreshold;
-        }
-        if (__syncthreads_or(over)) {
-            // raise each head's running max to max(m, tile max); rescale what was accumulated
-            tmem_ld16(tmem + lane_base + kTmemS + 16 * g, x);
+            tc_fence_after_sync();
+            const bool valid = (mask[(i & 3) * 4 + q] >> lane) & 1u;
+            float x[32];
+            tmem_ld32(s_cols, x);
             tmem_wait_ld();
+            bool over = false;
 #pragma unroll
-            for (int h = 0; h < 16; ++h) x[h] = valid ? x[h] * c : -INFINITY;
-            const float tmax = warp_transpose_reduce16<true>(x, lane);
-            if ((lane & 1) == 0) red[q * 64 + 16 * g + (lane >> 1)] = tmax;
-            __syncthreads();
-            if (tid < kHeads) {
-                const float tm = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
-                const float mo = head_m[tid];
-                const float mn = fmaxf(mo, tm);
-                head_alpha[tid] = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
-                head_m[tid] = mn;
+            for (int h = 0; h < 32; ++h) {
+                x[h] = valid ? x[h] * c : -INFINITY;
+                over |= (x[h] - head_m[32 * hh + h]) > kRescaleThreshold;
             }
-            __syncthreads();
-            if (i > 0) {
-                float al[16], o[16];
-#pragma unroll
-                for (int h = 0; h < 16; ++h) al[h] = head_alpha[16 * g + h];
-#pragma unroll 1
-                for (int cc = 0; cc < 5; ++cc) {  // 4 O^T chunks + the running sums
-                    const uint32_t col = (cc < 4 ? 64u * cc : kTmemL) + 16u * g;
-                    tmem_ld16(tmem + lane_base + col, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) o[h] *= al[h];
-                    tmem_st16(tmem + lane_base + col, o);
+            if (barrier_or(kBarIdSoftmax, kSoftmaxThreads, over)) {
+                // raise each head's running max to max(m, tile max); rescale what was accumulated
+                const float tmax = warp_transpose_reduce<true, 32>(x, lane);
+                red[q * 64 + 32 * hh + lane] = tmax;
+                named_barrier_sync(kBarIdSoftmax, kSoftmaxThreads);
+                if (tid < kHeads) {
+                    const float tm = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
+                    const float mo = head_m[tid];
+                    const float mn = fmaxf(mo, tm);
+                    head_alpha[tid] = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+                    head_m[tid] = mn;
                 }
-            }
-            tmem_ld16(tmem + lane_base + kTmemS + 16 * g, x);
-            tmem_wait_ld();
+                named_barrier_sync(kBarIdSoftmax, kSoftmaxThreads);
 #pragma unroll
-            for (int h = 0; h < 16; ++h) x[h] = valid ? fmaf(x[h], c, -head_m[16 * g + h]) : -INFINITY;
-        }
+                for (int h = 0; h < 32; ++h) l[h] *= head_alpha[32 * hh + h];
+                if (i > 0) {
+                    // the PV of tile i-1 is complete (the S^T commit of tile i covers it)
+#pragma unroll 1
+                    for (int part = 0; part < 8; ++part) {  // 4 chunks x 2 halves of 16 heads
+                        const int h0 = 32 * hh + 16 * (part & 1);
+                        const uint32_t col = tmem + lane_base + 64 * (part >> 1) + h0;
+                        float o[16];
+                        tmem_ld16(col, o);
+                        tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 16; ++h) x[h] = fast_exp2(x[h]);
-        {
-            float l[16];
-            if (i == 0) {
-#pragma unroll
-                for (int h = 0; h < 16; ++h) l[h] = x[h];
-            } else {
-                tmem_ld16(tmem + lane_base + kTmemL + 16 * g, l);
-                tmem_wait_ld();
-#pragma unroll
-                for (int h = 0; h < 16; ++h) l[h] += x[h];
-            }
-            tmem_st16(tmem + lane_base + kTmemL + 16 * g, l);
-        }
-        // P^T row r, heads 16g..16g+15: two 16-byte chunks of hi and two of lo
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float a0 = x[8 * half + 2 * j], a1 = x[8 * half + 2 * j + 1];
-                hw[j] = pack_bf16x2(a0, a1);
-                lw[j] = pack_bf16x2(a0 - __uint_as_float(hw[j] << 16), a1 - __uint_as_float(hw[j] & 0xFFFF0000u));
-            }
-            const uint32_t off = r * 128 + (((2 * g + half) ^ (r & 7)) << 4);
-            sts_v4(phi_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-            sts_v4(plo_s + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarPFull]);
-        tmem_wait_st();
-        tc_fence_before_sync();
-        __syncthreads();
-        // ---- 5. O^T += V^T.P^T
-        if (tid == 0) {
-            if (wait_phase(&bars[kBarPFull], i & 1, abort_flag, p)) {
-                tc_fence_after_sync();
-                const uint32_t acc0 = (i > 0) ? 1u : 0u;
-#pragma unroll
-                for (int mc = 0; mc < 4; ++mc) {
-                    const uint64_t a0 = dPV_a + static_cast<uint64_t>(mc * 2 * (kTile * 128 / 16));
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bh + ks * (2048 / 16), kIdescPV,
-                                    ks > 0 ? 1u : acc0);
-                        mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bl + ks * (2048 / 16), kIdescPV, 1u);
+                        for (int h = 0; h < 16; ++h) o[h] *= head_alpha[h0 + h];
+                        tmem_st16(col, o);
                     }
                 }
-                mma_commit(&bars[kBarPvDone]);
+                tmem_ld32(s_cols, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * c : -INFINITY;
             }
-        }
-        ok = warp_wait_phase(&bars[kBarPvDone], i & 1, abort_flag, p, lane);
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        tc_fence_after_sync();
-        // translation of tile i+2 completes into the buffer tile i used
-        if (tid < kTile && i + 2 < n) {
-            int code = -1;
-            if (idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks) {
-                if (page_next < 0 || static_cast<long long>(page_next) >= p.num_pages)
-                    atomicOr(p.err, SMLA_FLAG_BAD_PAGE);
-                else
-                    code = page_next * kPageTokens + (idx_next & (kPageTokens - 1));
+#pragma unroll
+            for (int h = 0; h < 32; ++h) {
+                x[h] = valid ? fast_exp2(x[h] - head_m[32 * hh + h]) : 0.0f;
+                l[h] += x[h];
             }
-            codes[buf * kTile + tid] = code;
-            idx_next = -1;
-            page_next = -1;
+            // P^T row r, heads 32hh..32hh+31: four 16-byte chunks of hi and four of lo
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a0 = x[8 * j + 2 * e], a1 = x[8 * j + 2 * e + 1];
+                    hw[e] = pack_bf16x2(a0, a1);
+                    lw[e] = pack_bf16x2(a0 - __uint_as_float(hw[e] << 16), a1 - __uint_as_float(hw[e] & 0xFFFF0000u));
+                }
+                const uint32_t off = r * 128 + (((4 * hh + j) ^ (r & 7)) << 4);
+                sts_v4(phi_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+                sts_v4(plo_s + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+            }
+            fence_proxy_async_smem();
+            tmem_wait_st();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kBarPFull]);
+            // warp 0's lane 0 issues PV of this tile and QK of the next one while the other
+            // softmax warps wait for that S^T
+            if (issuer && mma.pv(i) && i + 1 < n) mma.qk(i + 1);
+            __syncwarp();
         }
-        __syncthreads();
-    }
-
-    // every MMA issued above must be complete before tensor memory is released
-    if (tid == 0) {
-        if (spare_used) (void)mbar_wait(&bars[kBarSpare], 0, p.timeout_ns);
-        mma_commit(&bars[kBarDrain]);
-        (void)mbar_wait(&bars[kBarDrain], 0, p.timeout_ns);
-    }
-    __syncthreads();
-    const bool ok = !failed && !*abort_flag;
-
-    // ---- epilogue: per-head sums over the 128 token lanes, then O/l (or the cluster merge)
-    float l_part = 0.0f;
-    if (ok && n > 0) {
+        // the last PV is complete before the epilogue reads O^T
+        if (!failed && n > 0) {
+            const bool ok = warp_wait_phase(&bars[kBarKvFree + 3], (n - 1) & 1, abort_flag, p, lane);
+            (void)barrier_or(kBarIdSoftmax, kSoftmaxThreads, !ok);
+        }
+        // every MMA issued must be complete before tensor memory is released
+        if (issuer) mma.drain();
+        __syncwarp();
         tc_fence_after_sync();
-        float v[16];
-        tmem_ld16(tmem + lane_base + kTmemL + 16 * g, v);
-        tmem_wait_ld();
-        l_part = warp_transpose_reduce16<false>(v, lane);
+        const float ls = warp_transpose_reduce<false, 32>(l, lane);
+        red[q * 64 + 32 * hh + lane] = ls;
+    } else {
+        // ================================================================ producers
+        const int pt = tid - kSoftmaxThreads;
+        const uint32_t kv_s = smem_addr(sKV);
+        TileRegs tr;
+        if (n > 0) load_tile(pt, codes, p.cache, tr);
+        for (int i = 0; i < n; ++i) {
+            const int buf = i & 1;
+            // translation of tile i+2, first step: its topk indices
+            const int slot2 = (t_begin + i + 2) * kTile + pt;
+            int idx_next = -1;
+            if (pt < kTile && i + 2 < n && slot2 < p.topk) idx_next = __ldg(idx_row + slot2);
+            bool ok = produce_pair<0>(i, pt, lane, kv_s, bars, abort_flag, p, tr) &&
+                      produce_pair<1>(i, pt, lane, kv_s, bars, abort_flag, p, tr) &&
+                      produce_pair<2>(i, pt, lane, kv_s, bars, abort_flag, p, tr) &&
+                      produce_pair<3>(i, pt, lane, kv_s, bars, abort_flag, p, tr);
+            // second step: the block-table entries
+            int page_next = -1;
+            const bool in_range = idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks;
+            if (in_range) page_next = __ldg(bt_row + (idx_next >> 8));
+            // the rows of tile i+1 go in flight
+            if (ok && i + 1 < n) load_tile(pt, codes + (buf ^ 1) * kTile, p.cache, tr);
+            // tile i+2's codes replace tile i's (the loads above read the other buffer)
+            if (pt < kTile && i + 2 < n) {
+                int code = -1;
+                if (in_range) {
+                    if (page_next < 0 || static_cast<long long>(page_next) >= p.num_pages)
+                        atomicOr(p.err, SMLA_FLAG_BAD_PAGE);
+                    else
+                        code = page_next * kPageTokens + (idx_next & (kPageTokens - 1));
+                }
+                codes[buf * kTile + pt] = code;
+                const uint32_t bits = __ballot_sync(0xffffffffu, code >= 0);
+                if (lane == 0) mask[((i + 2) & 3) * 4 + (pt >> 5)] = bits;
+            }
+            if (barrier_or(kBarIdProducer, kProducerThreads, !ok)) break;
+        }
     }
-    if ((lane & 1) == 0) red[q * 64 + 16 * g + (lane >> 1)] = l_part;
+    tc_fence_before_sync();
     __syncthreads();
-    float *l_head = head_alpha;  // per-head sums for the epilogue
+    tc_fence_after_sync();
+    const bool ok = !*abort_flag;
+
+    // ---- epilogue: per-head sums (red holds them per TMEM quadrant), then O/l or the cluster merge
+    float *l_head = head_alpha;
     if (tid < kHeads) l_head[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
     __syncthreads();
     if (p.cluster_merge) {
-        cluster_epilogue(p, b, ok, n, tid, q, g, lane, tmem, lane_base, smem, &bars[kBarRecv], head_m, l_head, red);
+        cluster_epilogue(p, b, ok, n, tid, warp, lane, tmem, smem, &bars[kBarXch], head_m, l_head, red);
     } else if (ok) {
         if (tid < kHeads) {
             const float l = l_head[tid];
@@ -691,29 +778,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             else
                 p.part_lse[(static_cast<size_t>(b) * kHeads + tid) * p.nsplit + split] = val;
         }
-        float inv[16];
+        if (warp < kSoftmaxWarps) {
+            const int q = warp & 3;
+            const int hh = warp >> 2;
+            const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+            float inv[32];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
-            const float l = l_head[16 * g + h];
-            inv[h] = (l > 0.0f) ? 1.0f / l : 0.0f;
-        }
-#pragma unroll 1
-        for (int mc = 0; mc < 4; ++mc) {
-            float o[16];
-            if (n > 0) {
-                tmem_ld16(tmem + lane_base + 64 * mc + 16 * g, o);
-                tmem_wait_ld();
+            for (int h = 0; h < 32; ++h) {
+                const float l = l_head[32 * hh + h];
+                inv[h] = (l > 0.0f) ? 1.0f / l : 0.0f;
             }
-            const int d = 128 * mc + r;
-            if (p.nsplit == 1) {
-                float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * g) * kDim + d;
+#pragma unroll 1
+            for (int mc = 0; mc < 4; ++mc) {
+                float o[32];
+                if (n > 0) {
+                    tmem_ld32(tmem + lane_base + 64 * mc + 32 * hh, o);
+                    tmem_wait_ld();
+                }
+                const int d = 128 * mc + 32 * q + lane;
+                if (p.nsplit == 1) {
+                    float *dst = p.out + (static_cast<size_t>(b) * kHeads + 32 * hh) * kDim + d;
 #pragma unroll
-                for (int h = 0; h < 16; ++h) dst[h * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
-            } else {
-                float *dst = p.part_o + ((static_cast<size_t>(b) * kHeads + 16 * g) * p.nsplit + split) * kDim + d;
+                    for (int h = 0; h < 32; ++h) dst[h * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
+                } else {
+                    float *dst =
+                        p.part_o + ((static_cast<size_t>(b) * kHeads + 32 * hh) * p.nsplit + split) * kDim + d;
 #pragma unroll
-                for (int h = 0; h < 16; ++h)
-                    dst[static_cast<size_t>(h) * p.nsplit * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
+                    for (int h = 0; h < 32; ++h)
+                        dst[static_cast<size_t>(h) * p.nsplit * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
+                }
             }
         }
     }
@@ -904,16 +997,23 @@ bool sizes_ok(int B, int H, int topk) {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Up to this many splits of a request merge inside a thread-block cluster (through
-// distributed shared memory); beyond it they go through global partials and the
-// merge kernel.
+// Up to this many splits of a request merge inside a thread-block cluster (exchanging
+// through the workspace, ordered by the cluster barrier); beyond it they go through
+// normalised global partials and the merge kernel.
 constexpr int kMaxClusterSplits = 4;
 
+// Workspace after the header: nsplit == 1: nothing.  2..4 (cluster merge): the
+// (m, l) rows [B][nsplit][128] f32, then the exchanged O^T chunks
+// [B][4][nsplit-1][64][128] f32.  Above 4: part_lse [B][64][nsplit] f32, then
+// part_o [B][64][nsplit][512] f32.
 size_t workspace_for(int B, int topk, int nsplit) {
     size_t bytes = SMLA_WORKSPACE_HEADER;
     if (nsplit > kMaxClusterSplits) {
         const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
         bytes += round256(rows * sizeof(float)) + rows * SMLA_DIM * sizeof(float);
+    } else if (nsplit > 1) {
+        bytes += round256(static_cast<size_t>(B) * nsplit * 128 * sizeof(float)) +
+                 static_cast<size_t>(B) * 4 * (nsplit - 1) * 128 * SMLA_HEADS * sizeof(float);
     }
     (void)topk;
     return bytes;
@@ -988,7 +1088,8 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     p.lse = lse;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.err = reinterpret_cast<uint32_t *>(ws);
-    const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
+    const size_t rows = (nsplit > kMaxClusterSplits) ? static_cast<size_t>(B) * SMLA_HEADS * nsplit
+                                                             : static_cast<size_t>(B) * nsplit * 128;
     p.part_lse = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER);
     p.part_o = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER + round256(rows * sizeof(float)));
     p.num_pages = num_pages;
