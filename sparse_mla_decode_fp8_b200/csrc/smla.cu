@@ -85,10 +85,12 @@ constexpr int kSmemBytes = kSmemAbort + 4;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory limit");
 static_assert(kSmemBars % 8 == 0, "mbarriers need 8-byte alignment");
 
-// Tensor memory: O^T [0,256) (4 chunks of 128 dims x 64 heads), S^T buffers at 256 and 320.
+// Tensor memory: O^T [0,256) (4 chunks of 128 dims x 64 heads), S^T buffers at 256 and 320,
+// per-lane running sums L at 384 (lane = token of the tile, column = head).
 constexpr int kMlBytes = 128 * 4;  // one (m, l) row of the cluster merge
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;
+constexpr uint32_t kTmemL = 384;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, true, true);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(s - m) stays below 256 without a rescale
@@ -142,9 +144,8 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[N], int lane) 
 
 // Bounded wait on an mbarrier phase.  Gives up when another thread has aborted the
 // CTA or when `timeout_ns` passes (then it aborts the CTA and flags the error).
-__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                           const DecodeParams &p) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             const DecodeParams &p) {
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
@@ -155,6 +156,10 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volat
             return false;
         }
     }
+}
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                           const DecodeParams &p) {
+    return mbar_try_wait(bar, parity) || wait_phase_slow(bar, parity, abort_flag, p);
 }
 
 // Warp-uniform version: lane 0 waits, the verdict is broadcast, and every lane then
@@ -170,59 +175,26 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
 
 // ------------------------------------------------------------------ gather + dequant
 // The 128 x 36 sixteen-byte chunks of a tile are dealt out to the 256 producer threads
-// in four groups, one per K-block pair c (dims [128c, 128c+128)):
-//   pairs 0..2: 128 tokens x 8 nope chunks (16 dims)          -> 4 items per thread
-//   pair 3:     128 tokens x (4 nope + 8 rope chunks)          -> 6 items per thread
+// (pt) in four groups, one per K-block pair c (dims [128c, 128c+128)):
+//   pairs 0..2: chunk 8c + (pt & 7) of the tokens (pt >> 3) + 32u, u < 4     (nope)
+//   pair 3:     chunk 24 + (pt & 3) of the tokens (pt >> 2) + 64u, u < 2     (nope)
+//               chunk 28 + (pt & 7) of the tokens (pt >> 3) + 32u, u < 4     (rope)
 // Consecutive threads take consecutive chunks of a token row (coalesced loads).
-template <int C>
-struct PairShape {
-    static constexpr int kItems = (C < 3) ? 4 : 6;
-};
-
-template <int C>
-__device__ __forceinline__ void pair_item(int t, int u, int &r, int &chunk, int &kb, int &oc, bool &nope) {
-    const int j = t + kProducerThreads * u;
-    if constexpr (C < 3) {
-        r = j >> 3;
-        const int k = j & 7;
-        chunk = 8 * C + k;
-        kb = 2 * C + (k >> 2);
-        oc = 2 * (k & 3);
-        nope = true;
-    } else {
-        r = j / 12;
-        const int k = j - 12 * r;
-        if (k < 4) {
-            chunk = 24 + k;
-            kb = 6;
-            oc = 2 * k;
-            nope = true;
-        } else {
-            chunk = 28 + (k - 4);
-            kb = 7;
-            oc = k - 4;
-            nope = false;
-        }
-    }
-}
 
 // The FP8 bytes of one tile and their scales, held in registers between the load and
-// the dequantisation.  In pairs 0..2 a producer thread always takes chunk (pt & 7) of the
-// four tokens (pt >> 3) + 32u, so it loads each of those tokens' 8-byte scale row once
-// (srow[u]); in pair 3 it loads the one scale byte an item needs.
+// the dequantisation.  For pairs 0..2 each token's 8-byte scale row is loaded once.
 struct TileRegs {
-    uint4 raw0[4], raw1[4], raw2[4], raw3[6];
+    uint4 raw0[4], raw1[4], raw2[4], nope3[2], rope[4];
     uint2 srow[4];
-    uint32_t sc3[6];
+    uint32_t sc3[2];
 };
 
 __device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t *cache, TileRegs &tr) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        const int r = (t >> 3) + 32 * u;
+        const int code = codes[(t >> 3) + 32 * u];
         const int chunk = t & 7;
-        const int code = codes[r];
-        tr.raw0[u] = tr.raw1[u] = tr.raw2[u] = make_uint4(0u, 0u, 0u, 0u);
+        tr.raw0[u] = tr.raw1[u] = tr.raw2[u] = tr.rope[u] = make_uint4(0u, 0u, 0u, 0u);
         tr.srow[u] = make_uint2(0u, 0u);
         if (code >= 0) {
             const uint8_t *row = token_row(cache, code);
@@ -230,84 +202,73 @@ __device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t
             tr.raw1[u] = ld_stream_v4(row + (8 + chunk) * 16);
             tr.raw2[u] = ld_stream_v4(row + (16 + chunk) * 16);
             tr.srow[u] = ld_stream_v2(token_scales(cache, code));
+            tr.rope[u] = ld_stream_v4(row + (28 + chunk) * 16);
         }
     }
 #pragma unroll
-    for (int u = 0; u < 6; ++u) {
-        int r, chunk, kb, oc;
-        bool nope;
-        pair_item<3>(t, u, r, chunk, kb, oc, nope);
-        const int code = codes[r];
-        tr.raw3[u] = make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < 2; ++u) {
+        const int code = codes[(t >> 2) + 64 * u];
+        tr.nope3[u] = make_uint4(0u, 0u, 0u, 0u);
         tr.sc3[u] = 0u;
         if (code >= 0) {
-            tr.raw3[u] = ld_stream_v4(token_row(cache, code) + chunk * 16);
-            if (nope) tr.sc3[u] = ld_stream_u8(token_scales(cache, code) + (chunk >> 2));
+            tr.nope3[u] = ld_stream_v4(token_row(cache, code) + (24 + (t & 3)) * 16);
+            tr.sc3[u] = ld_stream_u8(token_scales(cache, code) + 6);
         }
     }
 }
 
-// Scale byte of item u of pair C (C < 3): byte 2C + ((t & 7) >> 2) of the token's scale row.
-template <int C>
-__device__ __forceinline__ uint32_t pair_scale(const TileRegs &tr, int t, int u) {
-    const int byte = 2 * C + ((t & 7) >> 2);
-    const uint32_t w = (byte < 4) ? tr.srow[u].x : tr.srow[u].y;
-    return (w >> (8 * (byte & 3))) & 0xFFu;
-}
-
-// Dequantises this thread's items of pair C into the swizzled bf16 tile (plain shared
-// stores; `kv` is the tile's shared-window address).
-template <int C>
-__device__ __forceinline__ void store_pair(int t, uint32_t kv, const TileRegs &tr) {
-#pragma unroll
-    for (int u = 0; u < PairShape<C>::kItems; ++u) {
-        int r, chunk, kb, oc;
-        bool nope;
-        pair_item<C>(t, u, r, chunk, kb, oc, nope);
-        const uint32_t row = kv + kb * (kTile * 128) + r * 128;
-        const int sw = r & 7;
-        uint4 raw;
-        uint32_t sc;
-        if constexpr (C == 0) {
-            raw = tr.raw0[u];
-            sc = pair_scale<C>(tr, t, u);
-        } else if constexpr (C == 1) {
-            raw = tr.raw1[u];
-            sc = pair_scale<C>(tr, t, u);
-        } else if constexpr (C == 2) {
-            raw = tr.raw2[u];
-            sc = pair_scale<C>(tr, t, u);
-        } else {
-            raw = tr.raw3[u];
-            sc = tr.sc3[u];
-        }
-        if (nope) {
-            uint4 lo, hi;
-            dequant16(raw, sc, lo, hi);
-            // odd K-blocks store their high half first so the 8 lanes of a store phase hit 8 bank groups
-            if ((kb & 1) == 0) {
-                sts_v4(row + ((oc ^ sw) << 4), lo);
-                sts_v4(row + (((oc + 1) ^ sw) << 4), hi);
-            } else {
-                sts_v4(row + (((oc + 1) ^ sw) << 4), hi);
-                sts_v4(row + ((oc ^ sw) << 4), lo);
-            }
-        } else {
-            sts_v4(row + ((oc ^ sw) << 4), raw);
-        }
+// Dequantises 16 e4m3 bytes (or copies 16 rope bytes) into row r of K-block kb of the
+// swizzled bf16 tile at 16-byte unit oc (two units for nope).
+__device__ __forceinline__ void store_item(uint32_t kv, int r, int kb, int oc, bool nope, const uint4 raw,
+                                           uint32_t sc) {
+    const uint32_t row = kv + kb * (kTile * 128) + r * 128;
+    const int sw = r & 7;
+    if (nope) {
+        uint4 lo, hi;
+        dequant16(raw, sc, lo, hi);
+        // odd K-blocks store their high half first so the 8 lanes of a store phase hit 8 bank groups
+        const bool odd = (kb & 1) != 0;
+        sts_v4(row + (((oc + (odd ? 1 : 0)) ^ sw) << 4), odd ? hi : lo);
+        sts_v4(row + (((oc + (odd ? 0 : 1)) ^ sw) << 4), odd ? lo : hi);
+    } else {
+        sts_v4(row + ((oc ^ sw) << 4), raw);
     }
 }
 
-// Producer step for pair C of a tile: wait until the PV of the previous tile has
-// released the pair, dequantise into it, publish it to the tensor core.
-template <int C>
-__device__ __forceinline__ bool produce_pair(int i, int pt, int lane, uint32_t kv_s, uint64_t *bars,
-                                             volatile int *abort_flag, const DecodeParams &p, const TileRegs &tr) {
-    if (i > 0 && !warp_wait_phase(&bars[kBarKvFree + C], (i - 1) & 1, abort_flag, p, lane)) return false;
-    store_pair<C>(pt, kv_s, tr);
-    fence_proxy_async_smem();  // this thread's stores -> visible to the tensor core
+// Publishes K-block pair c of the tile to the tensor core once this warp's stores are
+// visible to the async proxy.
+__device__ __forceinline__ void publish_pair(int c, int lane, uint64_t *bars) {
+    fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[kBarKvFull + C]);
+    if (lane == 0) mbar_arrive(&bars[kBarKvFull + c]);
+}
+
+// Producer steps for one tile: each K-block pair is dequantised as soon as the PV of the
+// previous tile has released it.  Pairs 0..2 share one rolled loop (in them a thread
+// takes chunk (pt & 7) of the tokens (pt >> 3) + 32u); pair 3 holds the last nope chunk
+// group and the rope.
+__device__ __forceinline__ bool produce_tile(int i, int pt, int lane, uint32_t kv_s, uint64_t *bars,
+                                             volatile int *abort_flag, const DecodeParams &p, const TileRegs &tr) {
+    const int k = pt & 7;
+#pragma unroll 1
+    for (int c = 0; c < 3; ++c) {
+        if (i > 0 && !warp_wait_phase(&bars[kBarKvFree + c], (i - 1) & 1, abort_flag, p, lane)) return false;
+        const int byte = 2 * c + (k >> 2);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint4 raw = (c == 0) ? tr.raw0[u] : (c == 1) ? tr.raw1[u] : tr.raw2[u];
+            const uint32_t w = (byte < 4) ? tr.srow[u].x : tr.srow[u].y;
+            store_item(kv_s, (pt >> 3) + 32 * u, 2 * c + (k >> 2), 2 * (k & 3), true, raw,
+                       (w >> (8 * (byte & 3))) & 0xFFu);
+        }
+        publish_pair(c, lane, bars);
+    }
+    if (i > 0 && !warp_wait_phase(&bars[kBarKvFree + 3], (i - 1) & 1, abort_flag, p, lane)) return false;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) store_item(kv_s, (pt >> 2) + 64 * u, 6, 2 * (pt & 3), true, tr.nope3[u], tr.sc3[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) store_item(kv_s, (pt >> 3) + 32 * u, 7, k, false, tr.rope[u], 0u);
+    publish_pair(3, lane, bars);
     return true;
 }
 
@@ -360,21 +321,22 @@ __device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool
     }
     if (worker) {
 #pragma unroll 1
-        for (int mc = 0; mc < 4; ++mc) {
+        for (int part = 0; part < 8; ++part) {  // 4 chunks x 2 halves of 16 heads
+            const int mc = part >> 1, h0 = 32 * hh + 16 * (part & 1);
             const int owner = mc % ns;
             if (owner == me) continue;
-            float o[32];
+            float o[16];
             if (live) {
-                tmem_ld32(tmem + lane_base + 64 * mc + 32 * hh, o);
+                tmem_ld16(tmem + lane_base + 64 * mc + h0, o);
                 tmem_wait_ld();
             } else {
 #pragma unroll
-                for (int h = 0; h < 32; ++h) o[h] = 0.0f;
+                for (int h = 0; h < 16; ++h) o[h] = 0.0f;
             }
             const int slot = (me < owner) ? me : me - 1;
-            float *dst = xch + ((mc * (ns - 1) + slot) * kHeads + 32 * hh) * 128 + d;
+            float *dst = xch + ((mc * (ns - 1) + slot) * kHeads + h0) * 128 + d;
 #pragma unroll
-            for (int h = 0; h < 32; ++h) __stcg(dst + h * 128, o[h]);
+            for (int h = 0; h < 16; ++h) __stcg(dst + h * 128, o[h]);
         }
     }
     fence_proxy_async_all();  // the peers read these rows and chunks with bulk copies
@@ -420,31 +382,31 @@ __device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool
     __syncthreads();
     if (!write || !worker) return;
 #pragma unroll 1
-    for (int lci = 0; lci < n_own; ++lci) {
-        const int mc = me + lci * ns;
-        float acc[32];
+    for (int part = 0; part < 2 * n_own; ++part) {  // owned chunks x 2 halves of 16 heads
+        const int lci = part >> 1, mc = me + lci * ns, h0 = 32 * hh + 16 * (part & 1);
+        float acc[16];
         if (live) {
-            tmem_ld32(tmem + lane_base + 64 * mc + 32 * hh, acc);
+            tmem_ld16(tmem + lane_base + 64 * mc + h0, acc);
             tmem_wait_ld();
         }
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-            const float w = weights[me * kHeads + 32 * hh + h];
+        for (int h = 0; h < 16; ++h) {
+            const float w = weights[me * kHeads + h0 + h];
             acc[h] = (live && w != 0.0f) ? acc[h] * w : 0.0f;
         }
         for (int s = 0; s < ns; ++s) {
             if (s == me) continue;
             const int slot = (s < me) ? s : s - 1;
-            const float *src = recv + ((lci * (ns - 1) + slot) * kHeads + 32 * hh) * 128 + d;
+            const float *src = recv + ((lci * (ns - 1) + slot) * kHeads + h0) * 128 + d;
 #pragma unroll
-            for (int h = 0; h < 32; ++h) {
-                const float w = weights[s * kHeads + 32 * hh + h];
+            for (int h = 0; h < 16; ++h) {
+                const float w = weights[s * kHeads + h0 + h];
                 if (w != 0.0f) acc[h] += src[h * 128] * w;
             }
         }
-        float *dst = p.out + (static_cast<size_t>(b) * kHeads + 32 * hh) * kDim + 128 * mc + d;
+        float *dst = p.out + (static_cast<size_t>(b) * kHeads + h0) * kDim + 128 * mc + d;
 #pragma unroll
-        for (int h = 0; h < 32; ++h) dst[h * kDim] = acc[h];
+        for (int h = 0; h < 16; ++h) dst[h * kDim] = acc[h];
     }
 }
 
@@ -474,18 +436,25 @@ struct MmaIssuer {
     __device__ void qk(int i) {
         if (!ok) return;
         const uint32_t s_col = tmem + kTmemS + 64 * (i & 1);
-#pragma unroll
+        uint64_t a = dQK_a, bq = dQK_b;
+        uint32_t acc = 0u;
+#pragma unroll 1
         for (int cp = 0; cp < 4; ++cp) {
             ok = ok && (i > 0 || cp > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
                  wait_phase(&bars[kBarKvFull + cp], i & 1, abort_flag, p);
             if (!ok) return;
             tc_fence_after_sync();
+#pragma unroll 1
+            for (int kb = 0; kb < 2; ++kb) {
+                // K-block: 4 MMAs of K=16 (32 bytes apart), the next K-block 16 KB (K) / 8 KB (Q) on
 #pragma unroll
-            for (int kb = 2 * cp; kb < 2 * cp + 2; ++kb)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(s_col, dQK_a + (kb * (kTile * 128) + kk * 32) / 16, dQK_b + (kb * 8192 + kk * 32) / 16,
-                                kIdescQK, (kb | kk) != 0);
+                for (int kk = 0; kk < 4; ++kk) {
+                    mma_bf16_ss(s_col, a + kk * 2, bq + kk * 2, kIdescQK, acc);
+                    acc = 1u;
+                }
+                a += (kTile * 128) / 16;
+                bq += 8192 / 16;
+            }
         }
         const bool hook = (i == 0) && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
         mma_commit(hook ? &bars[kBarSpare] : &bars[kBarSFull + (i & 1)]);
@@ -500,14 +469,19 @@ struct MmaIssuer {
         if (!ok) return false;
         tc_fence_after_sync();
         const uint32_t acc0 = (i > 0) ? 1u : 0u;
-#pragma unroll
+#pragma unroll 1
         for (int mc = 0; mc < 4; ++mc) {
-            const uint64_t a0 = dPV_a + static_cast<uint64_t>(mc * 2 * (kTile * 128 / 16));
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bh + ks * (2048 / 16), kIdescPV,
-                            ks > 0 ? 1u : acc0);
-                mma_bf16_ss(tmem + 64 * mc, a0 + ks * (2048 / 16), dPV_bl + ks * (2048 / 16), kIdescPV, 1u);
+            uint64_t a = dPV_a + static_cast<uint64_t>(mc * 2 * (kTile * 128 / 16));
+            uint64_t bh = dPV_bh, bl = dPV_bl;
+            uint32_t acc = acc0;
+#pragma unroll 2
+            for (int ks = 0; ks < 8; ++ks) {  // 16 tokens per step: 2 KB on in V^T and in P^T
+                mma_bf16_ss(tmem + 64 * mc, a, bh, kIdescPV, acc);
+                mma_bf16_ss(tmem + 64 * mc, a, bl, kIdescPV, 1u);
+                acc = 1u;
+                a += 2048 / 16;
+                bh += 2048 / 16;
+                bl += 2048 / 16;
             }
             mma_commit(&bars[kBarKvFree + mc]);
         }
@@ -623,13 +597,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         MmaIssuer mma(smem, tmem, p, bars, abort_flag);
         if (issuer && n > 0) mma.qk(0);
         __syncwarp();
-        float l[32];
-#pragma unroll
-        for (int h = 0; h < 32; ++h) l[h] = 0.0f;
         bool failed = false;
         for (int i = 0; i < n; ++i) {
             const int sb = i & 1;
             const uint32_t s_cols = tmem + lane_base + kTmemS + 64 * sb + 32 * hh;
+            const uint32_t l_cols = tmem + lane_base + kTmemL + 32 * hh;
             const bool ok = warp_wait_phase(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag, p, lane);
             if (barrier_or(kBarIdSoftmax, kSoftmaxThreads, !ok)) {
                 failed = true;
@@ -637,19 +609,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const bool valid = (mask[(i & 3) * 4 + q] >> lane) & 1u;
-            float x[32];
-            tmem_ld32(s_cols, x);
-            tmem_wait_ld();
+            // does any score exceed its head's running max by more than the threshold?
             bool over = false;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float x[16];
+                tmem_ld16(s_cols + 16 * half, x);
+                tmem_wait_ld();
+                const float *m = head_m + 32 * hh + 16 * half;
 #pragma unroll
-            for (int h = 0; h < 32; ++h) {
-                x[h] = valid ? x[h] * c : -INFINITY;
-                over |= (x[h] - head_m[32 * hh + h]) > kRescaleThreshold;
+                for (int h = 0; h < 16; ++h) over |= valid && (x[h] * c - m[h]) > kRescaleThreshold;
             }
             if (barrier_or(kBarIdSoftmax, kSoftmaxThreads, over)) {
                 // raise each head's running max to max(m, tile max); rescale what was accumulated
-                const float tmax = warp_transpose_reduce<true, 32>(x, lane);
-                red[q * 64 + 32 * hh + lane] = tmax;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float x[16];
+                    tmem_ld16(s_cols + 16 * half, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) x[h] = valid ? x[h] * c : -INFINITY;
+                    const float tmax = warp_transpose_reduce<true, 16>(x, lane);
+                    if ((lane & 1) == 0) red[q * 64 + 32 * hh + 16 * half + (lane >> 1)] = tmax;
+                }
                 named_barrier_sync(kBarIdSoftmax, kSoftmaxThreads);
                 if (tid < kHeads) {
                     const float tm = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
@@ -659,45 +641,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                     head_m[tid] = mn;
                 }
                 named_barrier_sync(kBarIdSoftmax, kSoftmaxThreads);
-#pragma unroll
-                for (int h = 0; h < 32; ++h) l[h] *= head_alpha[32 * hh + h];
                 if (i > 0) {
-                    // the PV of tile i-1 is complete (the S^T commit of tile i covers it)
+                    // the PV of tile i-1 is complete (the S^T commit of tile i covers it): rescale
+                    // the 4 O^T chunks and the sums, 16 heads at a time
 #pragma unroll 1
-                    for (int part = 0; part < 8; ++part) {  // 4 chunks x 2 halves of 16 heads
-                        const int h0 = 32 * hh + 16 * (part & 1);
-                        const uint32_t col = tmem + lane_base + 64 * (part >> 1) + h0;
+                    for (int part = 0; part < 10; ++part) {
+                        const int h0 = 16 * (part & 1);
+                        const uint32_t col = (part < 8 ? tmem + lane_base + 64 * (part >> 1) + 32 * hh : l_cols) + h0;
                         float o[16];
                         tmem_ld16(col, o);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < 16; ++h) o[h] *= head_alpha[h0 + h];
+                        for (int h = 0; h < 16; ++h) o[h] *= head_alpha[32 * hh + h0 + h];
                         tmem_st16(col, o);
                     }
                 }
-                tmem_ld32(s_cols, x);
+            }
+            // p = 2^(s c - m): add to the sums, write P^T row r as bf16 hi + lo
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float x[16], l[16];
+                tmem_ld16(s_cols + 16 * half, x);
+                if (i > 0) tmem_ld16(l_cols + 16 * half, l);
                 tmem_wait_ld();
+                const float *m = head_m + 32 * hh + 16 * half;
 #pragma unroll
-                for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * c : -INFINITY;
-            }
-#pragma unroll
-            for (int h = 0; h < 32; ++h) {
-                x[h] = valid ? fast_exp2(x[h] - head_m[32 * hh + h]) : 0.0f;
-                l[h] += x[h];
-            }
-            // P^T row r, heads 32hh..32hh+31: four 16-byte chunks of hi and four of lo
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a0 = x[8 * j + 2 * e], a1 = x[8 * j + 2 * e + 1];
-                    hw[e] = pack_bf16x2(a0, a1);
-                    lw[e] = pack_bf16x2(a0 - __uint_as_float(hw[e] << 16), a1 - __uint_as_float(hw[e] & 0xFFFF0000u));
+                for (int h = 0; h < 16; ++h) {
+                    x[h] = valid ? fast_exp2(x[h] * c - m[h]) : 0.0f;
+                    l[h] = (i > 0) ? l[h] + x[h] : x[h];
                 }
-                const uint32_t off = r * 128 + (((4 * hh + j) ^ (r & 7)) << 4);
-                sts_v4(phi_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-                sts_v4(plo_s + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+                tmem_st16(l_cols + 16 * half, l);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a0 = x[8 * j + 2 * e], a1 = x[8 * j + 2 * e + 1];
+                        hw[e] = pack_bf16x2(a0, a1);
+                        lw[e] = pack_bf16x2(a0 - __uint_as_float(hw[e] << 16), a1 - __uint_as_float(hw[e] & 0xFFFF0000u));
+                    }
+                    const uint32_t off = r * 128 + (((4 * hh + 2 * half + j) ^ (r & 7)) << 4);
+                    sts_v4(phi_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+                    sts_v4(plo_s + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+                }
             }
             fence_proxy_async_smem();
             tmem_wait_st();
@@ -718,8 +704,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (issuer) mma.drain();
         __syncwarp();
         tc_fence_after_sync();
-        const float ls = warp_transpose_reduce<false, 32>(l, lane);
-        red[q * 64 + 32 * hh + lane] = ls;
+        // per-head sums over this warp's 32 token lanes
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            float l[16];
+            if (n > 0 && !failed) {
+                tmem_ld16(tmem + lane_base + kTmemL + 32 * hh + 16 * half, l);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int h = 0; h < 16; ++h) l[h] = 0.0f;
+            }
+            const float ls = warp_transpose_reduce<false, 16>(l, lane);
+            if ((lane & 1) == 0) red[q * 64 + 32 * hh + 16 * half + (lane >> 1)] = ls;
+        }
     } else {
         // ================================================================ producers
         const int pt = tid - kSoftmaxThreads;
@@ -732,10 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot2 = (t_begin + i + 2) * kTile + pt;
             int idx_next = -1;
             if (pt < kTile && i + 2 < n && slot2 < p.topk) idx_next = __ldg(idx_row + slot2);
-            bool ok = produce_pair<0>(i, pt, lane, kv_s, bars, abort_flag, p, tr) &&
-                      produce_pair<1>(i, pt, lane, kv_s, bars, abort_flag, p, tr) &&
-                      produce_pair<2>(i, pt, lane, kv_s, bars, abort_flag, p, tr) &&
-                      produce_pair<3>(i, pt, lane, kv_s, bars, abort_flag, p, tr);
+            bool ok = produce_tile(i, pt, lane, kv_s, bars, abort_flag, p, tr);
             // second step: the block-table entries
             int page_next = -1;
             const bool in_range = idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks;
@@ -778,35 +773,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             else
                 p.part_lse[(static_cast<size_t>(b) * kHeads + tid) * p.nsplit + split] = val;
         }
+        if (tid < kHeads) {
+            const float l = l_head[tid];
+            red[tid] = (l > 0.0f) ? 1.0f / l : 0.0f;  // 1/l per head
+        }
+        __syncthreads();
         if (warp < kSoftmaxWarps) {
             const int q = warp & 3;
             const int hh = warp >> 2;
             const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-            float inv[32];
-#pragma unroll
-            for (int h = 0; h < 32; ++h) {
-                const float l = l_head[32 * hh + h];
-                inv[h] = (l > 0.0f) ? 1.0f / l : 0.0f;
-            }
+            // the nsplit > 1 partials are [b][head][split][dim]
+            const size_t head_stride = static_cast<size_t>(p.nsplit) * kDim;
+            float *base = (p.nsplit == 1) ? p.out + static_cast<size_t>(b) * kHeads * kDim
+                                          : p.part_o + static_cast<size_t>(b) * kHeads * head_stride + split * kDim;
 #pragma unroll 1
-            for (int mc = 0; mc < 4; ++mc) {
-                float o[32];
+            for (int part = 0; part < 8; ++part) {  // 4 chunks x 2 halves of 16 heads
+                const int mc = part >> 1, h0 = 32 * hh + 16 * (part & 1);
+                float o[16];
                 if (n > 0) {
-                    tmem_ld32(tmem + lane_base + 64 * mc + 32 * hh, o);
+                    tmem_ld16(tmem + lane_base + 64 * mc + h0, o);
                     tmem_wait_ld();
                 }
-                const int d = 128 * mc + 32 * q + lane;
-                if (p.nsplit == 1) {
-                    float *dst = p.out + (static_cast<size_t>(b) * kHeads + 32 * hh) * kDim + d;
+                float *dst = base + static_cast<size_t>(h0) * head_stride + 128 * mc + 32 * q + lane;
 #pragma unroll
-                    for (int h = 0; h < 32; ++h) dst[h * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
-                } else {
-                    float *dst =
-                        p.part_o + ((static_cast<size_t>(b) * kHeads + 32 * hh) * p.nsplit + split) * kDim + d;
-#pragma unroll
-                    for (int h = 0; h < 32; ++h)
-                        dst[static_cast<size_t>(h) * p.nsplit * kDim] = (n > 0) ? o[h] * inv[h] : 0.0f;
-                }
+                for (int h = 0; h < 16; ++h) dst[h * head_stride] = (n > 0) ? o[h] * red[h0 + h] : 0.0f;
             }
         }
     }

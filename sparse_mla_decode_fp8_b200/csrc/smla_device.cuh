@@ -73,6 +73,16 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_shifted(uint32_t two_bytes)
     return ((h2 >> 3) & 0x0FFF0FFFu) | (h2 & 0x80008000u);
 }
 
+// Scale bytes above 142: 2^(s-15) is not a bf16 normal, so multiply by 2^127 and then by
+// 2^(s-142); 0xFF gives NaN.  Out of line: such scales do not occur in normal caches.
+__device__ __noinline__ void scale_big(uint32_t (&o)[8], uint32_t s) {
+    const uint32_t big = 0x7F007F00u;                              // 2^127 in both halves
+    const uint32_t m = (s == 255u) ? 0x7FC0u : ((s - 15u) << 7);  // 2^(s-142) or NaN
+    const uint32_t m2 = m | (m << 16);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = bf16x2_mul(bf16x2_mul(o[i], big), m2);
+}
+
 // 16 e4m3 bytes with UE8M0 scale byte s -> 16 bf16 values e4m3 * 2^(s-127),
 // returned as two 16-byte chunks (dims 0-7, dims 8-15).  One bf16 multiply by
 // 2^(s-15) (two for s > 142, whose factor is not a bf16 normal); 0xFF gives NaN.
@@ -92,11 +102,7 @@ __device__ __forceinline__ void dequant16(const uint4 raw, const uint32_t s, uin
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] = bf16x2_mul(o[i], m2);
     } else {
-        const uint32_t big = 0x7F007F00u;                     // 2^127 in both halves
-        const uint32_t m = (s == 255u) ? 0x7FC0u : ((s - 15u) << 7);  // 2^(s-142) or NaN
-        const uint32_t m2 = m | (m << 16);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = bf16x2_mul(bf16x2_mul(o[i], big), m2);
+        scale_big(o, s);
     }
     lo = make_uint4(o[0], o[1], o[2], o[3]);
     hi = make_uint4(o[4], o[5], o[6], o[7]);
