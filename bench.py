@@ -332,13 +332,7 @@ def run_cuda(args):
     achieved_tf = units["flops"] / (call_ms * 1e-3) / 1e12
     t_hbm_us = units["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_tc_us = units["flops"] / (peaks["bf16_tflops"] * 1e12) * 1e6
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "decode_config4_traffic.json")
-    if os.path.exists(prof):
-        with open(prof) as f:
-            pj = json.load(f)
-        if pj.get("kernel_source_hash") == _kernel_hash():
-            traffic = pj.get("dram_bytes_per_launch")
+    traffic = _profiled_traffic()
     line = {
         "metric": METRIC, "value": job_throughput(world, B, topk, steps, max_ms), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step, "us_per_call": ms_step * 1e3,
@@ -368,6 +362,22 @@ def run_cuda(args):
         line["cpu_baseline"] = cpu_oracle_baseline(w, min_seconds=args.cpu_seconds, max_reps=200)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_config4.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for ln in f:
+            if ":" in ln and ln.split(":", 1)[0] in ("kernel_source_hash", "dram_bytes_per_launch"):
+                k, v = ln.split(":", 1)
+                fields[k] = v.strip()
+    if fields.get("kernel_source_hash") != _kernel_hash() or "dram_bytes_per_launch" not in fields:
+        return None
+    return int(fields["dram_bytes_per_launch"])
 
 
 def _kernel_hash() -> str:

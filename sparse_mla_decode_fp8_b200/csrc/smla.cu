@@ -93,7 +93,10 @@ constexpr uint32_t kTmemS = 256;
 constexpr uint32_t kTmemL = 384;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, true, true);
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(s - m) stays below 256 without a rescale
+// log2 units: the running max m of a head is raised (and O^T, the sums rescaled) only when a
+// score exceeds it by more than this, so p = 2^(s - m) stays below 2^24: P_hi + P_lo keep their
+// relative precision at any magnitude, and fp32 O^T sums of 2^24 x |v| stay far from overflow.
+constexpr float kRescaleThreshold = 24.0f;
 
 struct DecodeParams {
     const uint16_t *q;
@@ -140,6 +143,18 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[N], int lane) 
         return kMax ? fmaxf(v[0], got) : v[0] + got;
     }
     return v[0];
+}
+
+// 16 consecutive floats of shared memory (16-byte aligned) into registers.
+__device__ __forceinline__ void load16(const float *src, float (&v)[16]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 t = reinterpret_cast<const float4 *>(src)[j];
+        v[4 * j] = t.x;
+        v[4 * j + 1] = t.y;
+        v[4 * j + 2] = t.z;
+        v[4 * j + 3] = t.w;
+    }
 }
 
 // Bounded wait on an mbarrier phase.  Gives up when another thread has aborted the
@@ -616,7 +631,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float x[16];
                 tmem_ld16(s_cols + 16 * half, x);
                 tmem_wait_ld();
-                const float *m = head_m + 32 * hh + 16 * half;
+                float m[16];
+                load16(head_m + 32 * hh + 16 * half, m);
 #pragma unroll
                 for (int h = 0; h < 16; ++h) over |= valid && (x[h] * c - m[h]) > kRescaleThreshold;
             }
@@ -648,11 +664,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int part = 0; part < 10; ++part) {
                         const int h0 = 16 * (part & 1);
                         const uint32_t col = (part < 8 ? tmem + lane_base + 64 * (part >> 1) + 32 * hh : l_cols) + h0;
-                        float o[16];
+                        float o[16], al[16];
                         tmem_ld16(col, o);
+                        load16(head_alpha + 32 * hh + h0, al);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < 16; ++h) o[h] *= head_alpha[32 * hh + h0 + h];
+                        for (int h = 0; h < 16; ++h) o[h] *= al[h];
                         tmem_st16(col, o);
                     }
                 }
@@ -664,7 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld16(s_cols + 16 * half, x);
                 if (i > 0) tmem_ld16(l_cols + 16 * half, l);
                 tmem_wait_ld();
-                const float *m = head_m + 32 * hh + 16 * half;
+                float m[16];
+                load16(head_m + 32 * hh + 16 * half, m);
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     x[h] = valid ? fast_exp2(x[h] * c - m[h]) : 0.0f;
