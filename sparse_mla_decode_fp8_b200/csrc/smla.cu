@@ -1,7 +1,7 @@
 // smla.cu -- sparse MLA decode over an FP8 paged latent cache on B200 (sm_100a):
 // the decode kernel (gather -> dequant -> tcgen05 QK^T -> fp32 online softmax ->
-// tcgen05 PV), the split-K LSE-merge kernel, the gather debug kernel and the
-// C ABI declared in include/smla.h.
+// tcgen05 PV -> split-K merge), the split-K LSE-merge kernel, the gather debug
+// kernel and the C ABI declared in include/smla.h.
 //
 // Method ("The Turning Point: Architecting a Custom MMA Sparse-MLA Decode
 // Kernel"): one program per (request, topk split) handles all 64 heads, so each
@@ -9,26 +9,29 @@
 // run on tensor cores with fp32 accumulation, and split partials are merged by
 // their log-sum-exp (Step 5).
 //
-// B200 mapping, per CTA (one per SM, 512 threads in two warp roles):
-//   * Q[b] (64 heads x 512, bf16) stays in shared memory for the whole CTA (TMA).
-//   * Producer warps translate a tile of 128 topk slots through the block table,
-//     keep its FP8 rows in flight in registers (16-byte loads) while the previous
-//     tile is computed, and dequantise them into a bf16 [128 x 512] tile in the
-//     128-byte-swizzled layout the tensor core reads, one 128-dim K-block pair at
-//     a time as the previous tile's PV releases it.
+// B200 mapping, per CTA (one per SM, 16 worker warps + 1 control warp):
+//   * Q[b] (64 heads x 512, bf16) sits in shared memory (one TMA load) until the
+//     last score MMA; then that buffer receives the split merge's partials.
+//   * The worker warps hold the FP8 rows of the next 128-slot tile in registers
+//     (16-byte loads) while the rows of the tile after it are already on their
+//     way into L2 (bulk prefetches issued two tiles ahead), and dequantise a tile into a bf16 [128 x 512] buffer in the
+//     128-byte-swizzled layout the tensor core reads, one 128-dim chunk at a time
+//     as the previous tile's PV releases it.
 //   * S^T[128 tokens x 64 heads] = K_tile . Q^T: tcgen05.mma M=128 N=64, fp32 in
-//     tensor memory (two S^T buffers).  Tokens fill the 128-row M dimension, not
-//     the 64 heads.
-//   * Softmax warps (one thread per token lane and 32 heads) read S^T from tensor
-//     memory, keep the running max per head and the sums in registers, rescale
-//     O^T in tensor memory when the max grows, and write P^T as two bf16 terms
-//     (P = P_hi + P_lo).  One of their threads issues the MMAs.
-//   * O^T[512 x 64] += V^T . P^T with V = the same bf16 tile read MN-major:
-//     4 MMAs of M=128 per 16-token step, once with P_hi and once with P_lo, so P
-//     carries ~16 significant bits (a single bf16 P is not accurate enough when
-//     a few large latents dominate).
-//   * The epilogue reads O^T from tensor memory and writes O/l (or merges the
-//     splits of a request inside its cluster) and LSE = (m + log2 l) ln 2.
+//     tensor memory.  Tokens fill the 128-row M dimension, not the 64 heads.
+//   * The worker warps then read S^T from tensor memory (one token lane and 16
+//     heads per thread), keep the running max per head, rescale O^T in tensor
+//     memory when the max grows, and write P^T as two bf16 terms (P = P_hi + P_lo).
+//   * O^T[512 x 64] += V^T . P^T with V = the same bf16 tile read MN-major: 4 MMAs
+//     of M=128 per 16-token step, once with P_hi and once with P_lo, so P carries
+//     ~16 significant bits (a single bf16 P is not accurate enough when a few
+//     large latents dominate).
+//   * The control warp owns tensor memory and the mbarriers, loads Q and issues
+//     every MMA from one thread.
+//   * The epilogue writes O/l and LSE = (m + log2 l) ln 2, or, when the topk range
+//     of a request is split over a thread-block cluster, streams each CTA's O^T
+//     through distributed shared memory to the CTA that owns those output dims as
+//     soon as the last PV has finished that chunk.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -45,39 +48,43 @@
 
 namespace smla {
 
-constexpr int kTile = 128;                                  // topk slots per MMA tile (the M of S^T)
-constexpr int kSoftmaxWarps = 8;                            // warps 0..7: softmax and epilogue; warp 0 also
-                                                            // owns tensor memory and issues TMA and MMAs
-constexpr int kProducerWarps = 8;                           // warps 8..15: translation, gather, dequantisation
-constexpr int kThreads = 32 * (kSoftmaxWarps + kProducerWarps);  // 512: 128 registers per thread
-constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;         // 256
-constexpr int kProducerThreads = 32 * kProducerWarps;       // 256
-constexpr int kGatherThreads = 256;                         // threads of the gather debug kernel
-constexpr uint32_t kBarIdSoftmax = 1;                       // named barrier of the softmax warps
-constexpr uint32_t kBarIdProducer = 2;                      // named barrier of the producer warps
+constexpr int kTile = 128;                     // topk slots per MMA tile (the M of S^T)
+constexpr int kWorkerWarps = 16;               // gather, dequantisation, softmax, epilogue
+constexpr int kWorkers = 32 * kWorkerWarps;    // 512
+constexpr int kCtlWarp = kWorkerWarps;         // warp 16: tensor memory, mbarriers, TMA, MMA issue
+constexpr int kThreads = kWorkers + 32;        // 544 threads: at most 120 registers each
+constexpr int kGatherThreads = 256;            // threads of the gather debug kernel
+constexpr uint32_t kBarIdWorkers = 1;          // named barrier of the 512 worker threads
+constexpr uint32_t kBarIdHeads = 2;            // named barrier of worker threads 0..63 (one per head)
+constexpr int kWaiter = 32;                    // the worker that waits on behalf of all workers
+constexpr int kMaxClusterSplits = 4;           // splits of a request that merge inside a cluster
 
 // Dynamic shared memory map (bytes from a 1024-aligned base).
 constexpr int kSmemQ = 0;                         // 64 KB: 8 K-blocks x [64 heads x 128 B], TMA-written
 constexpr int kSmemKV = kSmemQ + 65536;           // 128 KB: 8 K-blocks x [128 tokens x 128 B]
 constexpr int kSmemPhi = kSmemKV + 131072;        // 16 KB: P_hi^T [128 tokens x 64 heads] bf16
 constexpr int kSmemPlo = kSmemPhi + 16384;        // 16 KB: P_lo^T
-constexpr int kSmemCodes = kSmemPlo + 16384;      // [2][128] int32 token codes (producers only)
-constexpr int kSmemMask = kSmemCodes + 1024;      // [4][4] u32: valid-token bits of a tile, ring of 4 tiles
+constexpr int kSmemCodes = kSmemPlo + 16384;      // [2][128] int32 token codes (tile ring)
+constexpr int kSmemRed = kSmemCodes + 1024;       // [4][64] f32: per-quadrant maxima or sums; merge weights
+constexpr int kSmemMask = kSmemRed + 1024;        // [4][4] u32: valid-token bits of a tile, ring of 4 tiles
 constexpr int kSmemHeadM = kSmemMask + 64;        // [64] running max per head (log2 units)
 constexpr int kSmemHeadAlpha = kSmemHeadM + 256;  // [64] rescale factor of the last max update; then the sums
-constexpr int kSmemRed = kSmemHeadAlpha + 256;    // [4][64] f32 cross-quadrant scratch
-constexpr int kSmemBars = kSmemRed + 1024;        // mbarriers (8 B each)
+constexpr int kSmemPeerLam = kSmemHeadAlpha + 256;  // [64] the other split's per-head log-sum-exp (2 splits)
+constexpr int kSmemBars = kSmemPeerLam + 256;     // mbarriers (8 B each)
 
 enum Bar : int {
-    kBarQ = 0,        // Q landed (TMA transaction bytes)
-    kBarKvFull = 1,   // + c (c = 0..3): K-block pair c of the tile written (8 producer-warp arrivals)
-    kBarKvFree = 5,   // + c: PV chunk c of the tile done (MMA commit): pair c may be overwritten
-    kBarSFull = 9,    // + s (s = 0..1): S^T buffer s complete (MMA commit)
-    kBarPFull = 11,   // P^T written (8 softmax-warp arrivals)
-    kBarDrain = 12,   // final commit before tensor memory is released
-    kBarSpare = 13,   // test hook target
-    kBarXch = 14,     // cluster merge: the other CTAs' rows and chunks landed (bulk-copy bytes)
-    kNumBars = 15,
+    kBarQ = 0,          // Q landed (TMA transaction bytes)
+    kBarKvFull = 1,     // + c (c = 0..3): dims chunk c of the tile written (16 worker-warp arrivals)
+    kBarKvFree = 5,     // + c: PV chunk c of the tile done (MMA commit): chunk c may be overwritten
+    kBarSFull = 9,      // + s (s = 0..1): S^T buffer s complete (MMA commit)
+    kBarPFull = 11,     // P^T written (16 worker-warp arrivals)
+    kBarDrain = 12,     // final commit before tensor memory is released
+    kBarSpare = 13,     // test hook target
+    kBarMl = 14,        // cluster merge: the peers' (m, l) rows are in (3-4 splits: the workspace, one arrival
+                        // per peer; 2 splits: the peer's log-sum-exp row, 256 transaction bytes)
+    kBarRxReady = 15,   // cluster merge: every peer's receive buffer is free (one arrival per peer)
+    kBarRx = 16,        // + k (k = 0..3): owned output unit k received (one arrival per sending lane)
+    kNumBars = 20,
 };
 constexpr int kSmemTmemSlot = kSmemBars + kNumBars * 8;
 constexpr int kSmemAbort = kSmemTmemSlot + 4;
@@ -86,17 +93,39 @@ static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory 
 static_assert(kSmemBars % 8 == 0, "mbarriers need 8-byte alignment");
 
 // Tensor memory: O^T [0,256) (4 chunks of 128 dims x 64 heads), S^T buffers at 256 and 320,
-// per-lane running sums L at 384 (lane = token of the tile, column = head).
-constexpr int kMlBytes = 128 * 4;  // one (m, l) row of the cluster merge
+// per-lane running sums L at 384 (lane = token row of the tile, column = head).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;
 constexpr uint32_t kTmemL = 384;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, true, true);
 // log2 units: the running max m of a head is raised (and O^T, the sums rescaled) only when a
-// score exceeds it by more than this, so p = 2^(s - m) stays below 2^24: P_hi + P_lo keep their
-// relative precision at any magnitude, and fp32 O^T sums of 2^24 x |v| stay far from overflow.
-constexpr float kRescaleThreshold = 24.0f;
+// score exceeds it by more than this, so p = 2^(s - m) stays below 2^64.  P_hi + P_lo keep
+// their relative precision at any magnitude, and fp32 sums of p x |v| over at most 2^16 slots
+// stay finite for |v| < 2^48.  A high threshold makes the rescale (two CTA barriers and a
+// pass over O^T in tensor memory) rare after the first tile, even when a few latents are
+// much larger than the rest.
+constexpr float kRescaleThreshold = 64.0f;
+
+// Split merge inside a cluster: the 512 output dims form 8 units of 64; unit u belongs
+// to CTA u % nsplit.  A CTA receives its units' partials from every peer into 16 KB
+// slots ([64 dims][64 heads] f32, 16-byte groups of 4 heads swizzled by dim & 7):
+// in the Q buffer (free after the last score MMA) when nsplit = 2, else in the KV
+// buffer (free after the last PV).
+constexpr int kUnitBytes = 64 * kHeads * 4;
+
+// The CTA's dynamic shared memory.  Every function addresses it through these
+// accessors (constant offsets from the shared window), so no 64-bit pointer to
+// shared memory has to live in a register.
+extern __shared__ __align__(1024) uint8_t g_smem[];
+__device__ __forceinline__ uint64_t *sm_bars() { return reinterpret_cast<uint64_t *>(g_smem + kSmemBars); }
+__device__ __forceinline__ int *sm_codes() { return reinterpret_cast<int *>(g_smem + kSmemCodes); }
+__device__ __forceinline__ uint32_t *sm_mask() { return reinterpret_cast<uint32_t *>(g_smem + kSmemMask); }
+__device__ __forceinline__ float *sm_head_m() { return reinterpret_cast<float *>(g_smem + kSmemHeadM); }
+__device__ __forceinline__ float *sm_head_alpha() { return reinterpret_cast<float *>(g_smem + kSmemHeadAlpha); }
+__device__ __forceinline__ float *sm_red() { return reinterpret_cast<float *>(g_smem + kSmemRed); }
+__device__ __forceinline__ volatile int *sm_abort() { return reinterpret_cast<volatile int *>(g_smem + kSmemAbort); }
+__device__ __forceinline__ float *sm_peer_lam() { return reinterpret_cast<float *>(g_smem + kSmemPeerLam); }
 
 struct DecodeParams {
     const uint16_t *q;
@@ -160,10 +189,12 @@ __device__ __forceinline__ void load16(const float *src, float (&v)[16]) {
 // Bounded wait on an mbarrier phase.  Gives up when another thread has aborted the
 // CTA or when `timeout_ns` passes (then it aborts the CTA and flags the error).
 __device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             const DecodeParams &p) {
+                                             const DecodeParams &p, uint32_t backoff_ns) {
     const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
+    for (uint32_t k = 1;; ++k) {
+        if (backoff_ns) __nanosleep(backoff_ns);
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((k & 31u) != 0) continue;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > p.timeout_ns) {
             *abort_flag = 1;
@@ -172,64 +203,129 @@ __device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, vol
         }
     }
 }
+// The MMA-issuing thread spins (backoff 0); waiting worker threads back off between
+// polls so they take few issue slots from the warps that share their scheduler.
+constexpr uint32_t kWorkerBackoffNs = 32;
 __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                           const DecodeParams &p) {
-    return mbar_try_wait(bar, parity) || wait_phase_slow(bar, parity, abort_flag, p);
+                                           const DecodeParams &p, uint32_t backoff_ns = 0) {
+    return mbar_test_wait(bar, parity) || wait_phase_slow(bar, parity, abort_flag, p, backoff_ns);
 }
 
-// Warp-uniform version: lane 0 waits, the verdict is broadcast, and every lane then
-// observes the completed phase itself (acquire) before touching the guarded data.
+// Warp-uniform version: lane 0 waits (acquire), the verdict is broadcast, and the warp
+// synchronisation orders the other lanes after its observation.
 __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                 const DecodeParams &p, int lane) {
     int ok = 1;
-    if (lane == 0) ok = wait_phase(bar, parity, abort_flag, p) ? 1 : 0;
+    if (lane == 0) ok = wait_phase(bar, parity, abort_flag, p, kWorkerBackoffNs) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (ok) (void)mbar_try_wait(bar, parity);
+    __syncwarp();
     return ok != 0;
 }
 
-// ------------------------------------------------------------------ gather + dequant
-// The 128 x 36 sixteen-byte chunks of a tile are dealt out to the 256 producer threads
-// (pt) in four groups, one per K-block pair c (dims [128c, 128c+128)):
-//   pairs 0..2: chunk 8c + (pt & 7) of the tokens (pt >> 3) + 32u, u < 4     (nope)
-//   pair 3:     chunk 24 + (pt & 3) of the tokens (pt >> 2) + 64u, u < 2     (nope)
-//               chunk 28 + (pt & 7) of the tokens (pt >> 3) + 32u, u < 4     (rope)
-// Consecutive threads take consecutive chunks of a token row (coalesced loads).
+// Bounded wait on a phase completed by other CTAs of the cluster (acquire at cluster
+// scope); every calling thread observes the phase itself.
+__device__ __noinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parity, const DecodeParams &p) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t k = 1;; ++k) {
+        if (mbar_test_wait_cluster(bar, parity)) return true;
+        __nanosleep(kWorkerBackoffNs);
+        if ((k & 31u) == 0 && global_timer_ns() - t0 > p.timeout_ns) {
+            atomicOr(p.err, SMLA_FLAG_TIMEOUT);
+            return false;
+        }
+    }
+}
 
-// The FP8 bytes of one tile and their scales, held in registers between the load and
-// the dequantisation.  For pairs 0..2 each token's 8-byte scale row is loaded once.
-struct TileRegs {
-    uint4 raw0[4], raw1[4], raw2[4], nope3[2], rope[4];
-    uint2 srow[4];
-    uint32_t sc3[2];
+// Worker-wide waits: one worker thread (in warp 1, so it does not share a scheduler
+// with the MMA-issuing warp 16) waits on the mbarrier phase, with acquire semantics,
+// while the other workers block in a named barrier; the barrier then orders every
+// worker after that observation (the others do not poll the mbarrier word, which would
+// serialise 512 accesses to one address).  `enabled` false skips the wait but keeps
+// the barrier (every worker calls these with the same arguments).  Returns false if
+// the wait failed or was skipped.
+__device__ __forceinline__ bool workers_wait(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
+                                             bool enabled = true) {
+    bool ok = enabled;
+    if (t == kWaiter && enabled) ok = wait_phase(bar, parity, sm_abort(), p, kWorkerBackoffNs);
+    return !barrier_or(kBarIdWorkers, kWorkers, !ok);
+}
+__device__ __forceinline__ bool workers_wait_cluster(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
+                                                     bool enabled = true) {
+    bool ok = enabled;
+    if (t == kWaiter && enabled) ok = wait_cluster_phase(bar, parity, p);
+    return !barrier_or(kBarIdWorkers, kWorkers, !ok);
+}
+
+// ------------------------------------------------------------------ gather + dequant
+// A tile's 128 token rows are dealt out to the 512 worker threads t, 9 sixteen-byte
+// chunks each, grouped by dims chunk c (dims [128c, 128c+128)):
+//   chunks 0..2: nope chunk 8c + (t & 7) of the tokens (t >> 3) and (t >> 3) + 64
+//   chunk 3:     nope chunk 24 + (t & 3) of the token t >> 2, and rope chunk
+//                28 + (t & 7) of the tokens (t >> 3) and (t >> 3) + 64
+// Consecutive threads take consecutive chunks of a token row (coalesced loads).
+// A Slot holds those bytes and their UE8M0 scales in registers between the load and
+// the dequantisation.
+struct Slot {
+    uint4 raw[3][2];  // nope chunks of dims chunks 0..2, tokens (t >> 3) + 64u
+    uint4 rope[2];    // rope chunk of the same tokens
+    uint4 nope3;      // nope chunk 24 + (t & 3) of token t >> 2
+    uint2 srow[2];    // scale rows of tokens (t >> 3) + 64u
+    uint32_t sc3;     // scale byte 6 of token t >> 2
 };
 
-__device__ __forceinline__ void load_tile(int t, const int *codes, const uint8_t *cache, TileRegs &tr) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int code = codes[(t >> 3) + 32 * u];
-        const int chunk = t & 7;
-        tr.raw0[u] = tr.raw1[u] = tr.raw2[u] = tr.rope[u] = make_uint4(0u, 0u, 0u, 0u);
-        tr.srow[u] = make_uint2(0u, 0u);
-        if (code >= 0) {
-            const uint8_t *row = token_row(cache, code);
-            tr.raw0[u] = ld_stream_v4(row + chunk * 16);
-            tr.raw1[u] = ld_stream_v4(row + (8 + chunk) * 16);
-            tr.raw2[u] = ld_stream_v4(row + (16 + chunk) * 16);
-            tr.srow[u] = ld_stream_v2(token_scales(cache, code));
-            tr.rope[u] = ld_stream_v4(row + (28 + chunk) * 16);
-        }
-    }
+// The loads of one dims chunk's items of a tile (part 0..3), so that a tile's rows can
+// go in flight chunk by chunk as the registers of the previous tile's chunk free up.
+// Part 2 also loads the scale rows (their last use is chunk 2), part 3 the rest.
+__device__ __forceinline__ void load_part(int part, int t, const int *codes, const uint8_t *cache, Slot &s) {
+    const int k8 = t & 7;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        const int code = codes[(t >> 2) + 64 * u];
-        tr.nope3[u] = make_uint4(0u, 0u, 0u, 0u);
-        tr.sc3[u] = 0u;
+        const int code = codes[(t >> 3) + 64 * u];
+        const uint8_t *row = token_row(cache, code >= 0 ? code : 0);
+        if (part == 0) s.raw[0][u] = (code >= 0) ? ld_stream_v4(row + k8 * 16) : make_uint4(0u, 0u, 0u, 0u);
+        if (part == 1) s.raw[1][u] = (code >= 0) ? ld_stream_v4(row + (8 + k8) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        if (part == 2) {
+            s.raw[2][u] = (code >= 0) ? ld_stream_v4(row + (16 + k8) * 16) : make_uint4(0u, 0u, 0u, 0u);
+            s.srow[u] = (code >= 0) ? ld_stream_v2(token_scales(cache, code)) : make_uint2(0u, 0u);
+        }
+        if (part == 3) s.rope[u] = (code >= 0) ? ld_stream_v4(row + (28 + k8) * 16) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (part == 3) {
+        const int code3 = codes[t >> 2];
+        s.nope3 = (code3 >= 0) ? ld_stream_v4(token_row(cache, code3) + (24 + (t & 3)) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        s.sc3 = (code3 >= 0) ? ld_stream_u8(token_scales(cache, code3) + 6) : 0u;
+    }
+}
+
+__device__ __forceinline__ void load_slot(int t, const int *codes, const uint8_t *cache, Slot &s) {
+    const int k8 = t & 7;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int code = codes[(t >> 3) + 64 * u];
+        s.raw[0][u] = s.raw[1][u] = s.raw[2][u] = s.rope[u] = make_uint4(0u, 0u, 0u, 0u);
+        s.srow[u] = make_uint2(0u, 0u);
         if (code >= 0) {
-            tr.nope3[u] = ld_stream_v4(token_row(cache, code) + (24 + (t & 3)) * 16);
-            tr.sc3[u] = ld_stream_u8(token_scales(cache, code) + 6);
+            const uint8_t *row = token_row(cache, code);
+            s.raw[0][u] = ld_stream_v4(row + k8 * 16);
+            s.raw[1][u] = ld_stream_v4(row + (8 + k8) * 16);
+            s.raw[2][u] = ld_stream_v4(row + (16 + k8) * 16);
+            s.rope[u] = ld_stream_v4(row + (28 + k8) * 16);
+            s.srow[u] = ld_stream_v2(token_scales(cache, code));
         }
     }
+    const int code3 = codes[t >> 2];
+    s.nope3 = make_uint4(0u, 0u, 0u, 0u);
+    s.sc3 = 0u;
+    if (code3 >= 0) {
+        s.nope3 = ld_stream_v4(token_row(cache, code3) + (24 + (t & 3)) * 16);
+        s.sc3 = ld_stream_u8(token_scales(cache, code3) + 6);
+    }
+}
+
+// Asks L2 to fetch a token's row and scale row ahead of the register loads.
+__device__ __forceinline__ void prefetch_token_l2(const uint8_t *cache, int code) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], 576;" ::"l"(token_row(cache, code)) : "memory");
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(token_scales(cache, code)) : "memory");
 }
 
 // Dequantises 16 e4m3 bytes (or copies 16 rope bytes) into row r of K-block kb of the
@@ -250,307 +346,581 @@ __device__ __forceinline__ void store_item(uint32_t kv, int r, int kb, int oc, b
     }
 }
 
-// Publishes K-block pair c of the tile to the tensor core once this warp's stores are
+// Publishes dims chunk c of the tile to the tensor core once this warp's stores are
 // visible to the async proxy.
-__device__ __forceinline__ void publish_pair(int c, int lane, uint64_t *bars) {
+__device__ __forceinline__ void publish_chunk(int c, int lane, uint64_t *bars) {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[kBarKvFull + c]);
 }
 
-// Producer steps for one tile: each K-block pair is dequantised as soon as the PV of the
-// previous tile has released it.  Pairs 0..2 share one rolled loop (in them a thread
-// takes chunk (pt & 7) of the tokens (pt >> 3) + 32u); pair 3 holds the last nope chunk
-// group and the rope.
-__device__ __forceinline__ bool produce_tile(int i, int pt, int lane, uint32_t kv_s, uint64_t *bars,
-                                             volatile int *abort_flag, const DecodeParams &p, const TileRegs &tr) {
-    const int k = pt & 7;
+// Dequantisation of tile i: each dims chunk is written as soon as the PV of tile i-1
+// has released it, and its registers then take the same chunk's rows of tile i+1
+// (`next`, null for the last tile): the load issue, which stalls while the memory
+// pipeline is full, overlaps the waits for the PV instead of delaying the softmax.
+__device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const DecodeParams &p, Slot &s,
+                                             const int *next) {
+    const uint32_t kv = smem_addr(g_smem + kSmemKV);
+    uint64_t *bars = sm_bars();
+    const int k8 = t & 7;
 #pragma unroll 1
     for (int c = 0; c < 3; ++c) {
-        if (i > 0 && !warp_wait_phase(&bars[kBarKvFree + c], (i - 1) & 1, abort_flag, p, lane)) return false;
-        const int byte = 2 * c + (k >> 2);
+        if (i > 0 && !workers_wait(&bars[kBarKvFree + c], (i - 1) & 1, p, t)) return false;
+        const int kb = 2 * c + (k8 >> 2);  // also the scale group of these 16 dims
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const uint4 raw = (c == 0) ? tr.raw0[u] : (c == 1) ? tr.raw1[u] : tr.raw2[u];
-            const uint32_t w = (byte < 4) ? tr.srow[u].x : tr.srow[u].y;
-            store_item(kv_s, (pt >> 3) + 32 * u, 2 * c + (k >> 2), 2 * (k & 3), true, raw,
-                       (w >> (8 * (byte & 3))) & 0xFFu);
+        for (int u = 0; u < 2; ++u) {
+            const uint4 raw = (c == 0) ? s.raw[0][u] : (c == 1) ? s.raw[1][u] : s.raw[2][u];
+            const uint32_t w = (kb < 4) ? s.srow[u].x : s.srow[u].y;
+            store_item(kv, (t >> 3) + 64 * u, kb, 2 * (k8 & 3), true, raw, (w >> (8 * (kb & 3))) & 0xFFu);
         }
-        publish_pair(c, lane, bars);
+        publish_chunk(c, lane, bars);
+        if (next) load_part(c, t, next, p.cache, s);
     }
-    if (i > 0 && !warp_wait_phase(&bars[kBarKvFree + 3], (i - 1) & 1, abort_flag, p, lane)) return false;
+    if (i > 0 && !workers_wait(&bars[kBarKvFree + 3], (i - 1) & 1, p, t)) return false;
+    store_item(kv, t >> 2, 6, 2 * (t & 3), true, s.nope3, s.sc3);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) store_item(kv_s, (pt >> 2) + 64 * u, 6, 2 * (pt & 3), true, tr.nope3[u], tr.sc3[u]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) store_item(kv_s, (pt >> 3) + 32 * u, 7, k, false, tr.rope[u], 0u);
-    publish_pair(3, lane, bars);
+    for (int u = 0; u < 2; ++u) store_item(kv, (t >> 3) + 64 * u, 7, k8, false, s.rope[u], 0u);
+    publish_chunk(3, lane, bars);
+    if (next) load_part(3, t, next, p.cache, s);
     return true;
 }
 
-// ------------------------------------------------------------------ split merge in a cluster
-// The nsplit (2..4) CTAs of one request form a thread-block cluster, which makes them
-// co-resident.  After the last PV, CTA s holds un-normalised O^T_s (tensor memory), its
-// per-head running max m_s (log2 units) and sum l_s.  With L = log2 sum_s 2^(m_s) l_s,
-// the merged output is O = sum_s 2^(m_s - L) O^T_s and LSE = L ln 2 (the split-K
-// log-sum-exp merge).  Output dims are dealt out by 128-dim chunk: chunk mc belongs to
-// CTA mc % nsplit.  Each CTA publishes its (m_s, l_s) row and the O^T_s chunks it does
-// not own to the workspace (coalesced stores that stay in L2); after one cluster barrier
-// (release / acquire) each owner pulls what it needs into its own shared memory with
-// bulk copies counted on one mbarrier (a single L2 round trip), then merges.
-// Distributed shared memory is not used for the exchange: its per-SM bandwidth is a
-// fraction of what L2 gives one SM.
-//   ml   [B][nsplit][m(64) | l(64)] f32
-//   xch  [B][4 chunks][nsplit - 1 sender slots][64 heads][128 dims] f32 (a warp's
-//        32 consecutive dims are one 128-byte line); the sender slot of CTA s in
-//        chunk mc is s, minus one when s is above the owner.
-// Shared memory (the operand buffers are dead by then): the rows at the Q buffer
-// [nsplit][128] f32, the received chunks at the KV buffer [owned chunk][sender slot]
-// [64][128] f32.
-// Called by every thread of the CTA (the cluster barrier needs them all); the softmax
-// warps (quadrant q, head half hh) do the work.
-constexpr int kXchBlock = kHeads * 128 * 4;  // one 128-dim chunk of O^T, bytes
+// ------------------------------------------------------------------ MMA issue
+// The tensor-core side of the pipeline, run by one thread of the control warp, with
+// every descriptor in registers and each chunk's MMAs unrolled: a single thread issues
+// all of them, so instructions between two MMAs directly slow the tensor core.  Every
+// wait is bounded; a failed wait stops the issue.
+//
+// Descriptor words (128-byte swizzle, see sw128_desc): the high word holds SBO = 1024
+// (8 rows of 128 bytes), the version and the swizzle mode; the low word holds the
+// address (16-byte units) and LBO.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
 
-__device__ __noinline__ void cluster_epilogue(const DecodeParams &p, int b, bool ok, int n, int tid, int warp,
-                                              int lane, uint32_t tmem, uint8_t *smem, uint64_t *bar_xch,
-                                              const float *head_m, const float *l_head, float *weights) {
-    const int ns = p.nsplit;
-    const int me = static_cast<int>(cluster_ctarank());
-    const int n_own = (4 - me + ns - 1) / ns;  // chunks me, me + ns, ... below 4
-    const bool worker = warp < kSoftmaxWarps;
-    const int q = warp & 3, hh = (warp >> 2) & 1;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    const int d = 32 * q + lane;  // row of O^T within a chunk
-    const bool live = ok && n > 0;
-    float *ml = p.part_lse + static_cast<size_t>(b) * ns * 128;
-    float *xch = p.part_o + static_cast<size_t>(b) * 4 * (ns - 1) * (kHeads * 128);
-    float *ml_s = reinterpret_cast<float *>(smem + kSmemQ);
-    const float *recv = reinterpret_cast<const float *>(smem + kSmemKV);
-
-    if (tid < kHeads) {
-        const float mv = live ? head_m[tid] : -INFINITY;
-        const float lv = live ? l_head[tid] : 0.0f;
-        ml[me * 128 + tid] = mv;
-        ml[me * 128 + 64 + tid] = lv;
-        ml_s[me * 128 + tid] = mv;
-        ml_s[me * 128 + 64 + tid] = lv;
-    }
-    if (worker) {
-#pragma unroll 1
-        for (int part = 0; part < 8; ++part) {  // 4 chunks x 2 halves of 16 heads
-            const int mc = part >> 1, h0 = 32 * hh + 16 * (part & 1);
-            const int owner = mc % ns;
-            if (owner == me) continue;
-            float o[16];
-            if (live) {
-                tmem_ld16(tmem + lane_base + 64 * mc + h0, o);
-                tmem_wait_ld();
-            } else {
+// S^T += K.Q^T over dims chunk cp: 2 K-blocks x 4 steps of K = 16 (the K rows are
+// 128 bytes per K-block, K-blocks 16 KB apart; Q K-blocks 8 KB apart).
+__device__ __forceinline__ void issue_qk_chunk(uint32_t d, uint32_t a_lo, uint32_t b_lo, bool first) {
+    if (first)
+        mma_bf16_ss(d, desc_from(a_lo, kDescHi), desc_from(b_lo, kDescHi), kIdescQK, 0u);
+    else
+        mma_bf16_ss_acc(d, desc_from(a_lo, kDescHi), desc_from(b_lo, kDescHi), kIdescQK);
 #pragma unroll
-                for (int h = 0; h < 16; ++h) o[h] = 0.0f;
-            }
-            const int slot = (me < owner) ? me : me - 1;
-            float *dst = xch + ((mc * (ns - 1) + slot) * kHeads + h0) * 128 + d;
-#pragma unroll
-            for (int h = 0; h < 16; ++h) __stcg(dst + h * 128, o[h]);
-        }
-    }
-    fence_proxy_async_all();  // the peers read these rows and chunks with bulk copies
-    // every CTA's row and chunks are written before any owner fetches them
-    cluster_sync();
-    int got = 1;
-    if (tid == 0) {
-        fence_proxy_async_all();
-        mbar_arrive_expect_tx(bar_xch, (ns - 1) * (kMlBytes + n_own * kXchBlock));
-        for (int s = 0; s < ns; ++s) {
-            if (s == me) continue;
-            bulk_load(ml_s + s * 128, ml + s * 128, kMlBytes, bar_xch);
-            const int slot = (s < me) ? s : s - 1;
-            for (int lci = 0; lci < n_own; ++lci) {
-                const int mc = me + lci * ns;
-                bulk_load(smem + kSmemKV + (lci * (ns - 1) + slot) * kXchBlock,
-                          xch + (mc * (ns - 1) + slot) * (kHeads * 128), kXchBlock, bar_xch);
-            }
-        }
-        got = mbar_wait(bar_xch, 0, p.timeout_ns) ? 1 : 0;
-        if (!got) atomicOr(p.err, SMLA_FLAG_TIMEOUT);
-    }
-    got = __syncthreads_and(got);
-    if (got) (void)mbar_try_wait(bar_xch, 0);  // every thread observes the completed phase
-    const bool write = ok && got;
-    if (tid < kHeads) {
-        float mx = -INFINITY;
-        for (int s = 0; s < ns; ++s)
-            if (ml_s[s * 128 + 64 + tid] > 0.0f) mx = fmaxf(mx, ml_s[s * 128 + tid]);
-        float sum = 0.0f;
-        for (int s = 0; s < ns; ++s) {
-            const float lv = ml_s[s * 128 + 64 + tid];
-            if (lv > 0.0f) sum += exp2f(ml_s[s * 128 + tid] - mx) * lv;
-        }
-        const float L = (sum > 0.0f) ? mx + log2f(sum) : -INFINITY;
-        for (int s = 0; s < ns; ++s) {
-            const float lv = ml_s[s * 128 + 64 + tid];
-            weights[s * kHeads + tid] = (sum > 0.0f && lv > 0.0f) ? exp2f(ml_s[s * 128 + tid] - L) : 0.0f;
-        }
-        if (me == 0 && write)
-            p.lse[static_cast<size_t>(b) * kHeads + tid] = (sum > 0.0f) ? L * 0.69314718055994531f : -INFINITY;
-    }
-    __syncthreads();
-    if (!write || !worker) return;
-#pragma unroll 1
-    for (int part = 0; part < 2 * n_own; ++part) {  // owned chunks x 2 halves of 16 heads
-        const int lci = part >> 1, mc = me + lci * ns, h0 = 32 * hh + 16 * (part & 1);
-        float acc[16];
-        if (live) {
-            tmem_ld16(tmem + lane_base + 64 * mc + h0, acc);
-            tmem_wait_ld();
-        }
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-            const float w = weights[me * kHeads + h0 + h];
-            acc[h] = (live && w != 0.0f) ? acc[h] * w : 0.0f;
-        }
-        for (int s = 0; s < ns; ++s) {
-            if (s == me) continue;
-            const int slot = (s < me) ? s : s - 1;
-            const float *src = recv + ((lci * (ns - 1) + slot) * kHeads + h0) * 128 + d;
-#pragma unroll
-            for (int h = 0; h < 16; ++h) {
-                const float w = weights[s * kHeads + h0 + h];
-                if (w != 0.0f) acc[h] += src[h * 128] * w;
-            }
-        }
-        float *dst = p.out + (static_cast<size_t>(b) * kHeads + h0) * kDim + 128 * mc + d;
-#pragma unroll
-        for (int h = 0; h < 16; ++h) dst[h * kDim] = acc[h];
+    for (int k = 1; k < 8; ++k) {
+        const uint32_t ao = (k >> 2) * ((kTile * 128) >> 4) + (k & 3) * 2;
+        const uint32_t bo = (k >> 2) * (8192 >> 4) + (k & 3) * 2;
+        mma_bf16_ss_acc(d, desc_from(a_lo + ao, kDescHi), desc_from(b_lo + bo, kDescHi), kIdescQK);
     }
 }
 
-// ------------------------------------------------------------------ MMA issue
-// The tensor-core side of the pipeline, run by one thread.  Every wait is bounded; a
-// failed wait leaves `ok` false and issues nothing more.
-struct MmaIssuer {
-    uint64_t dQK_a, dQK_b, dPV_a, dPV_bh, dPV_bl;
-    uint32_t tmem;
-    const DecodeParams &p;
-    uint64_t *bars;
-    volatile int *abort_flag;
-    bool ok = true;
-    bool spare_used = false;
-
-    __device__ MmaIssuer(uint8_t *smem, uint32_t tmem_, const DecodeParams &p_, uint64_t *bars_,
-                         volatile int *abort_)
-        : tmem(tmem_), p(p_), bars(bars_), abort_flag(abort_) {
-        dQK_a = sw128_desc(smem_addr(smem + kSmemKV), 16, 1024);
-        dQK_b = sw128_desc(smem_addr(smem + kSmemQ), 16, 1024);
-        dPV_a = sw128_desc(smem_addr(smem + kSmemKV), kTile * 128, 1024);
-        dPV_bh = sw128_desc(smem_addr(smem + kSmemPhi), 8192, 1024);
-        dPV_bl = sw128_desc(smem_addr(smem + kSmemPlo), 8192, 1024);
-    }
-
-    // S^T[tile i] = K.Q^T into buffer i&1, one K-block pair as soon as it is published.
-    __device__ void qk(int i) {
-        if (!ok) return;
-        const uint32_t s_col = tmem + kTmemS + 64 * (i & 1);
-        uint64_t a = dQK_a, bq = dQK_b;
-        uint32_t acc = 0u;
-#pragma unroll 1
-        for (int cp = 0; cp < 4; ++cp) {
-            ok = ok && (i > 0 || cp > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
-                 wait_phase(&bars[kBarKvFull + cp], i & 1, abort_flag, p);
-            if (!ok) return;
-            tc_fence_after_sync();
-#pragma unroll 1
-            for (int kb = 0; kb < 2; ++kb) {
-                // K-block: 4 MMAs of K=16 (32 bytes apart), the next K-block 16 KB (K) / 8 KB (Q) on
+// O^T chunk += V^T.P_hi^T + V^T.P_lo^T over the tile's 128 tokens: 8 steps of 16 tokens
+// (2 KB apart in the MN-major V^T and P^T).
+__device__ __forceinline__ void issue_pv_chunk(uint32_t d, uint32_t a_lo, uint32_t bh_lo, uint32_t bl_lo,
+                                               bool accumulate) {
+    if (accumulate)
+        mma_bf16_ss_acc(d, desc_from(a_lo, kDescHi), desc_from(bh_lo, kDescHi), kIdescPV);
+    else
+        mma_bf16_ss(d, desc_from(a_lo, kDescHi), desc_from(bh_lo, kDescHi), kIdescPV, 0u);
+    mma_bf16_ss_acc(d, desc_from(a_lo, kDescHi), desc_from(bl_lo, kDescHi), kIdescPV);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    mma_bf16_ss(s_col, a + kk * 2, bq + kk * 2, kIdescQK, acc);
-                    acc = 1u;
-                }
-                a += (kTile * 128) / 16;
-                bq += 8192 / 16;
-            }
+    for (int ks = 1; ks < 8; ++ks) {
+        const uint32_t o = ks * (2048 >> 4);
+        mma_bf16_ss_acc(d, desc_from(a_lo + o, kDescHi), desc_from(bh_lo + o, kDescHi), kIdescPV);
+        mma_bf16_ss_acc(d, desc_from(a_lo + o, kDescHi), desc_from(bl_lo + o, kDescHi), kIdescPV);
+    }
+}
+
+// For each tile i: S^T = K.Q^T into buffer i&1 chunk by chunk as the workers publish the
+// tile's dims chunks, then, once every worker has written P^T, O^T += V^T.P^T with a
+// commit per 128-dim chunk (freeing that chunk of the tile buffer; in the last tile it
+// makes that chunk of O^T final).
+__device__ __forceinline__ void mma_issue_loop(uint32_t tmem, const DecodeParams &p, int n) {
+    uint64_t *bars = sm_bars();
+    volatile int *abort_flag = sm_abort();
+    const uint32_t kv = smem_addr(g_smem + kSmemKV);
+    const uint32_t qk_a = desc_lo(kv, 16), qk_b = desc_lo(smem_addr(g_smem + kSmemQ), 16);
+    const uint32_t pv_a = desc_lo(kv, kTile * 128);
+    const uint32_t pv_bh = desc_lo(smem_addr(g_smem + kSmemPhi), 8192);
+    const uint32_t pv_bl = desc_lo(smem_addr(g_smem + kSmemPlo), 8192);
+    bool ok = true, spare_used = false;
+    for (int i = 0; i < n && ok; ++i) {
+        const uint32_t s_col = tmem + kTmemS + 64 * (i & 1);
+#pragma unroll 1
+        for (int cp = 0; cp < 4 && ok; ++cp) {
+            ok = (i > 0 || cp > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
+                 wait_phase(&bars[kBarKvFull + cp], i & 1, abort_flag, p);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_qk_chunk(s_col, qk_a + cp * 2 * ((kTile * 128) >> 4), qk_b + cp * 2 * (8192 >> 4), cp == 0);
         }
+        if (!ok) break;
         const bool hook = (i == 0) && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
         mma_commit(hook ? &bars[kBarSpare] : &bars[kBarSFull + (i & 1)]);
         spare_used = spare_used || hook;
-    }
-
-    // O^T += V^T.P_hi^T + V^T.P_lo^T of tile i once every softmax warp has written P^T;
-    // each 128-dim chunk is committed to the producers as it completes.
-    __device__ bool pv(int i) {
-        if (!ok) return false;
         ok = wait_phase(&bars[kBarPFull], i & 1, abort_flag, p);
-        if (!ok) return false;
+        if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t acc0 = (i > 0) ? 1u : 0u;
 #pragma unroll 1
         for (int mc = 0; mc < 4; ++mc) {
-            uint64_t a = dPV_a + static_cast<uint64_t>(mc * 2 * (kTile * 128 / 16));
-            uint64_t bh = dPV_bh, bl = dPV_bl;
-            uint32_t acc = acc0;
-#pragma unroll 2
-            for (int ks = 0; ks < 8; ++ks) {  // 16 tokens per step: 2 KB on in V^T and in P^T
-                mma_bf16_ss(tmem + 64 * mc, a, bh, kIdescPV, acc);
-                mma_bf16_ss(tmem + 64 * mc, a, bl, kIdescPV, 1u);
-                acc = 1u;
-                a += 2048 / 16;
-                bh += 2048 / 16;
-                bl += 2048 / 16;
-            }
+            issue_pv_chunk(tmem + 64 * mc, pv_a + mc * 2 * ((kTile * 128) >> 4), pv_bh, pv_bl, i > 0);
             mma_commit(&bars[kBarKvFree + mc]);
         }
+    }
+    // every MMA issued must be complete before tensor memory is released
+    if (spare_used) (void)mbar_wait(&bars[kBarSpare], 0, p.timeout_ns);
+    mma_commit(&bars[kBarDrain]);
+    (void)mbar_wait(&bars[kBarDrain], 0, p.timeout_ns);
+}
+
+// ------------------------------------------------------------------ worker state
+// Per-thread view of the CTA for the worker warps.  Warp w reads tensor-memory lanes
+// 32q.. (q = w & 3: the tokens 32q..32q+31 of S^T, or dims 32q.. of an O^T chunk)
+// and the 16 heads 16hq.. (hq = w >> 2).
+struct Worker {
+    const DecodeParams &p;
+    uint32_t tmem;
+    int t, warp, lane, q, hq;
+    uint32_t lane_base;
+
+    // Softmax of tile i: p = 2^(s c - m) against the running max m, which is raised (with
+    // a rescale of O^T and of the sums) only when a score exceeds it by more than
+    // kRescaleThreshold; P^T is written as bf16 hi + lo terms.
+    __device__ __forceinline__ bool softmax(int i) {
+        const int sb = i & 1;
+        if (!workers_wait(&sm_bars()[kBarSFull + sb], (i >> 1) & 1, p, t)) return false;
+        tc_fence_after_sync();
+        const float c = p.scale_log2;
+        const bool valid = (sm_mask()[(i & 3) * 4 + q] >> lane) & 1u;
+        const uint32_t s_col = tmem + lane_base + kTmemS + 64 * sb + 16 * hq;
+        const float4 *hm4 = reinterpret_cast<const float4 *>(sm_head_m() + 16 * hq);
+        // does any score exceed its head's running max by more than the threshold?
+        bool over = false;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float x[8];
+            tmem_ld8(s_col + 8 * half, x);
+            const float4 m0 = hm4[2 * half], m1 = hm4[2 * half + 1];
+            const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 8; ++h) over |= valid && (x[h] * c - mm[h]) > kRescaleThreshold;
+        }
+        if (barrier_or(kBarIdWorkers, kWorkers, over)) rescale(i, valid, s_col);
+        // p = 2^(s c - m): add to the sums, write P^T row r as bf16 hi + lo, 8 heads at a time
+        const int r = 32 * q + lane;
+        const uint32_t phi = smem_addr(g_smem + kSmemPhi), plo = smem_addr(g_smem + kSmemPlo);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t l_col = tmem + lane_base + kTmemL + 16 * hq + 8 * half;
+            float x[8], l[8];
+            tmem_ld8(s_col + 8 * half, x);
+            if (i > 0) tmem_ld8(l_col, l);
+            const float4 m0 = hm4[2 * half], m1 = hm4[2 * half + 1];
+            const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+            tmem_wait_ld();
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float a[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int h = 2 * e + k;
+                    a[k] = valid ? fast_exp2(x[h] * c - mm[h]) : 0.0f;
+                    l[h] = (i > 0) ? l[h] + a[k] : a[k];
+                }
+                // hi = the top 16 bits of p (exact bf16), lo = bf16(p - hi): ~16 significant bits
+                hw[e] = pack_bf16x2_trunc(a[0], a[1]);
+                lw[e] = pack_bf16x2(a[0] - __uint_as_float(hw[e] << 16), a[1] - __uint_as_float(hw[e] & 0xFFFF0000u));
+            }
+            tmem_st8(l_col, l);
+            const uint32_t off = r * 128 + (((2 * hq + half) ^ (r & 7)) << 4);
+            sts_v4(phi + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+            sts_v4(plo + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm_bars()[kBarPFull]);
         return true;
     }
 
-    __device__ void drain() {
-        if (spare_used) (void)mbar_wait(&bars[kBarSpare], 0, p.timeout_ns);
-        mma_commit(&bars[kBarDrain]);
-        (void)mbar_wait(&bars[kBarDrain], 0, p.timeout_ns);
+    // Raises each head's running max to max(m, tile max) and rescales what was
+    // accumulated (O^T and the sums) by 2^(m_old - m_new).  Rare: the max moves only
+    // past kRescaleThreshold, and on the first tile with a valid token.
+    __device__ __noinline__ void rescale(int i, bool valid, uint32_t s_col) {
+        const float c = p.scale_log2;
+        float y[16];
+        tmem_ld16(s_col, y);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 16; ++h) y[h] = valid ? y[h] * c : -INFINITY;
+        const float tmax = warp_transpose_reduce<true, 16>(y, lane);
+        if ((lane & 1) == 0) sm_red()[q * 64 + 16 * hq + (lane >> 1)] = tmax;
+        named_barrier_sync(kBarIdWorkers, kWorkers);
+        if (t < kHeads) {
+            const float *red = sm_red();
+            const float tm = fmaxf(fmaxf(red[t], red[64 + t]), fmaxf(red[128 + t], red[192 + t]));
+            const float mo = sm_head_m()[t];
+            const float mn = fmaxf(mo, tm);
+            sm_head_alpha()[t] = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+            sm_head_m()[t] = mn;
+        }
+        named_barrier_sync(kBarIdWorkers, kWorkers);
+        if (i == 0) return;  // nothing accumulated yet
+        // the PV of tile i-1 is complete (the S^T commit of tile i covers it): rescale the
+        // 4 O^T chunks and the sums, unless none of this warp's 16 heads moved
+        float al[16];
+        load16(sm_head_alpha() + 16 * hq, al);
+        bool moved = false;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) moved |= al[h] != 1.0f;
+        if (!moved) return;
+#pragma unroll 1
+        for (int mc = 0; mc < 5; ++mc) {
+            const uint32_t col = tmem + lane_base + (mc < 4 ? 64 * mc : kTmemL) + 16 * hq;
+            float o[16];
+            tmem_ld16(col, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h) o[h] *= al[h];
+            tmem_st16(col, o);
+        }
+        tmem_wait_st();
+    }
+
+    // Per-head sums over all 128 token lanes into the head_alpha array (every worker calls it;
+    // `have` is false when no tile was completed, the sums are then zero).
+    __device__ __forceinline__ void reduce_sums(bool have) {
+        float v[16];
+        if (have) {
+            tmem_ld16(tmem + lane_base + kTmemL + 16 * hq, v);
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int h = 0; h < 16; ++h) v[h] = 0.0f;
+        }
+        const float s = warp_transpose_reduce<false, 16>(v, lane);
+        if ((lane & 1) == 0) sm_red()[q * 64 + 16 * hq + (lane >> 1)] = s;
+        named_barrier_sync(kBarIdWorkers, kWorkers);
+        if (t < kHeads) sm_head_alpha()[t] = (sm_red()[t] + sm_red()[64 + t]) + (sm_red()[128 + t] + sm_red()[192 + t]);
+        named_barrier_sync(kBarIdWorkers, kWorkers);
     }
 };
 
+// One step of the worker pipeline for tile i: dequantise it from the register slot while
+// refilling the slot with tile i+1 (from L2: its rows were prefetched one step earlier,
+// at kernel entry for tile 1), run the softmax of tile i, then translate tile i+2 and
+// prefetch its rows.
+// Translation runs two tiles ahead in stages so no thread waits on a dependent load:
+// the topk index of a slot is loaded one step before its block-table entry, which is
+// loaded before the token code is formed (threads t < 128 own slot t of every tile).
+struct Translator {
+    int idx_a = -1;   // topk index of slot t of tile i+2
+    int idx_b = -1;   // of tile i+3
+    int page_a = -1;  // block-table entry for idx_a
+};
+
+__device__ __forceinline__ int slot_index(const DecodeParams &p, int t_begin, int tile, int t) {
+    return (t_begin + tile) * kTile + t;
+}
+
+__device__ __forceinline__ bool worker_step(Worker &w, int i, int n, int t_begin, int seq_len, const int32_t *bt_row,
+                                            const int32_t *idx_row, Translator &tr, Slot &cur) {
+    const DecodeParams &p = w.p;
+    const int t = w.t;
+    if (t < kTile && i + 2 < n) {
+        tr.page_a = slot_in_range(tr.idx_a, seq_len, p.max_blocks) ? __ldg(bt_row + (tr.idx_a >> 8)) : -1;
+        const int s3 = slot_index(p, t_begin, i + 3, t);
+        tr.idx_b = (i + 3 < n && s3 < p.topk) ? __ldg(idx_row + s3) : -1;
+    }
+    const int *next = (i + 1 < n) ? sm_codes() + ((i + 1) & 1) * kTile : nullptr;
+    if (!dequant_tile(i, t, w.lane, p, cur, next)) return false;  // uniform over the workers
+    if (!w.softmax(i)) return false;
+    if (t < kTile && i + 2 < n) {
+        // tile i's codes are dead (its rows were loaded one step ago): tile i+2 takes the buffer
+        const int code = slot_in_range(tr.idx_a, seq_len, p.max_blocks)
+                             ? slot_code(tr.idx_a, tr.page_a, p.num_pages, p.err)
+                             : -1;
+        sm_codes()[(i & 1) * kTile + t] = code;
+        const uint32_t bits = __ballot_sync(0xffffffffu, code >= 0);
+        if (w.lane == 0) sm_mask()[((i + 2) & 3) * 4 + (t >> 5)] = bits;
+        if (code >= 0) prefetch_token_l2(p.cache, code);
+    }
+    tr.idx_a = tr.idx_b;
+    return true;
+}
+
+// ------------------------------------------------------------------ epilogues
+// Writes dims chunk c of this CTA's O^T, each head h scaled by scale[h] (16 heads 16hq..,
+// in registers), to dst + h * head_stride + 128c + dim with 16-byte accesses: the warp
+// stages its 16 heads x 32 dims through the (dead) Q buffer as [head][dim] rows, then
+// every lane writes 4 consecutive dims of a head (plain stores, or atomic adds into an
+// output the splits share).  What is written: kChunkTmem the scaled O^T, kChunkZero zeros
+// (no tile, or weight 0), kChunkNan NaN (a failed wait: the result is invalid).
+enum ChunkSource : int { kChunkNan = 0, kChunkZero = 1, kChunkTmem = 2 };
+__device__ __forceinline__ void write_chunk(const Worker &w, int c, const float (&scale)[16], float *dst,
+                                            size_t head_stride, int source, bool add) {
+    float v[16];
+    if (source == kChunkTmem) {
+        tmem_ld16(w.tmem + w.lane_base + 64 * c + 16 * w.hq, v);
+        tmem_wait_ld();
+    }
+    float *stage = reinterpret_cast<float *>(g_smem + kSmemQ);  // [64 heads][128 dims] f32
+#pragma unroll
+    for (int h = 0; h < 16; ++h)
+        stage[(16 * w.hq + h) * 128 + 32 * w.q + w.lane] =
+            (source == kChunkTmem) ? v[h] * scale[h] : (source == kChunkZero) ? 0.0f : NAN;
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int h = 16 * w.hq + 4 * k + (w.lane >> 3);
+        const int d = 32 * w.q + 4 * (w.lane & 7);
+        const float4 x = *reinterpret_cast<const float4 *>(stage + h * 128 + d);
+        float *o = dst + static_cast<size_t>(h) * head_stride + 128 * c + d;
+        if (add)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o), "f"(x.x), "f"(x.y), "f"(x.z),
+                         "f"(x.w)
+                         : "memory");
+        else
+            *reinterpret_cast<float4 *>(o) = x;
+    }
+    __syncwarp();
+}
+
+// nsplit = 1: O = O^T / l and LSE; nsplit > 4: normalised partials for the merge
+// kernel.  A CTA that aborted writes NaN (its rows are then visibly invalid).
+__device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int n, bool ok) {
+    const DecodeParams &p = w.p;
+    if (n > 0) ok = workers_wait(&sm_bars()[kBarKvFree + 3], (n - 1) & 1, p, w.t, ok);
+    float *inv = sm_red();
+    if (w.t < kHeads) {
+        const float l = sm_head_alpha()[w.t];
+        const float val = !ok ? NAN : (l > 0.0f) ? (sm_head_m()[w.t] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.nsplit == 1)
+            p.lse[static_cast<size_t>(b) * kHeads + w.t] = val;
+        else
+            p.part_lse[(static_cast<size_t>(b) * kHeads + w.t) * p.nsplit + split] = val;
+        inv[w.t] = !ok ? NAN : (l > 0.0f) ? 1.0f / l : 0.0f;
+    }
+    named_barrier_sync(kBarIdWorkers, kWorkers);
+    // the nsplit > 1 partials are [b][head][split][dim]
+    const size_t head_stride = static_cast<size_t>(p.nsplit) * kDim;
+    float *base = (p.nsplit == 1) ? p.out + static_cast<size_t>(b) * kHeads * kDim
+                                  : p.part_o + static_cast<size_t>(b) * kHeads * head_stride + split * kDim;
+    float sc[16];
+    load16(inv + 16 * w.hq, sc);
+    const int source = !ok ? kChunkNan : (n > 0) ? kChunkTmem : kChunkZero;
+#pragma unroll 1
+    for (int mc = 0; mc < 4; ++mc) write_chunk(w, mc, sc, base, head_stride, source, false);
+}
+
+// nsplit = 2 in one cluster.  With lambda_s = m_s + log2 l_s (the log-sum-exp of split s
+// in log2 units) and L = log2(2^lambda_0 + 2^lambda_1), the merged output is
+// O = sum_s 2^(lambda_s - L) O^T_s / l_s and LSE = L ln 2 (the split-K log-sum-exp
+// merge).  Each CTA sends its 64 lambdas to the other (asynchronous stores into a row
+// kept for them, counted as transaction bytes on the receiver's mbarrier), and, chunk
+// by chunk as its last PV finishes, adds its scaled O^T into the output, which both
+// CTAs zeroed half of at entry (two terms: the sum does not depend on their order).
+__device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) {
+    const DecodeParams &p = w.p;
+    const int me = static_cast<int>(cluster_ctarank());
+    const int t = w.t;
+    uint64_t *bars = sm_bars();
+    float lam = NAN;
+    if (t < kHeads) {
+        const float l = sm_head_alpha()[t];
+        lam = !ok ? NAN : (n > 0 && l > 0.0f) ? sm_head_m()[t] + log2f(l) : -INFINITY;
+        const uint32_t dst = map_to_rank(sm_peer_lam() + t, me ^ 1);
+        const uint32_t bar = map_to_rank(&bars[kBarMl], me ^ 1);
+        asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst),
+                     "r"(__float_as_uint(lam)), "r"(bar)
+                     : "memory");
+    }
+    const bool got = workers_wait(&bars[kBarMl], 0, p, t);
+    float *scale = sm_red();
+    if (t < kHeads) {
+        const float other = got ? sm_peer_lam()[t] : NAN;
+        const float mx = fmaxf(lam, other);
+        const bool bad = isnan(lam) || isnan(other);
+        const float L = (mx == -INFINITY) ? -INFINITY : mx + log2f(exp2f(lam - mx) + exp2f(other - mx));
+        const float l = sm_head_alpha()[t];
+        scale[t] = bad ? NAN : (lam == -INFINITY) ? 0.0f : exp2f(lam - L) / l;
+        if (me == 0) p.lse[static_cast<size_t>(b) * kHeads + t] = bad ? NAN : L * 0.69314718055994531f;
+    }
+    named_barrier_sync(kBarIdWorkers, kWorkers);
+    float sc[16];
+    load16(scale + 16 * w.hq, sc);
+    float *base = p.out + static_cast<size_t>(b) * kHeads * kDim;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        const bool chunk_ok = workers_wait(&bars[kBarKvFree + c], (n - 1) & 1, p, t, ok && n > 0);
+        // a split without tiles adds zeros; a failed wait NaN
+        const int source = chunk_ok ? kChunkTmem : (ok && n == 0) ? kChunkZero : kChunkNan;
+        write_chunk(w, c, sc, base, kDim, source, true);
+    }
+}
+
+// nsplit = 3..4 in one cluster.  With L = log2 sum_s 2^(m_s) l_s over the splits s, the
+// merged output is O = sum_s 2^(m_s - L) O^T_s and LSE = L ln 2 (the split-K
+// log-sum-exp merge).  Every CTA publishes its (m, l) row to the workspace and signals
+// its peers; output unit u (dims [64u, 64u+64)) belongs to CTA u % nsplit.  Chunk by
+// chunk, as the last PV finishes dims chunk c, the warps whose lanes cover a unit of
+// chunk c (u = 2c + q/2) that another CTA owns store their O^T values into the owner's
+// receive slot (distributed shared memory) and signal it with one arrival per lane;
+// the owner warps wait for every peer's values of their unit and write the merged
+// output.
+__device__ __forceinline__ void epilogue_cluster(Worker &w, int b, int n, bool ok) {
+    const DecodeParams &p = w.p;
+    const int ns = p.nsplit;
+    const int me = static_cast<int>(cluster_ctarank());
+    const int t = w.t;
+    uint64_t *bars = sm_bars();
+    float *ml = p.part_lse + static_cast<size_t>(b) * ns * 128;
+    const int rx_base = (ns == 2) ? kSmemQ : kSmemKV;
+    // 1. publish (m, l) (one arrival per peer once all 64 heads are stored); signal that
+    //    this CTA's receive buffer is free: with nsplit = 2 it is the Q buffer, idle since
+    //    the last score MMA (the softmax of the last tile waited for it), otherwise the KV
+    //    buffer once the last PV is done
+    if (t < kHeads) {
+        __stcg(ml + me * 128 + t, ok ? sm_head_m()[t] : NAN);
+        __stcg(ml + me * 128 + 64 + t, ok ? sm_head_alpha()[t] : NAN);
+        fence_acq_rel_cluster();
+        named_barrier_sync(kBarIdHeads, kHeads);
+        if (t == 0) {
+            for (int s = 0; s < ns; ++s)
+                if (s != me) mbar_arrive_remote(map_to_rank(&bars[kBarMl], s));
+            if (ns > 2 && ok && n > 0) (void)wait_phase(&bars[kBarKvFree + 3], (n - 1) & 1, sm_abort(), p);
+            for (int s = 0; s < ns; ++s)
+                if (s != me) mbar_arrive_remote(map_to_rank(&bars[kBarRxReady], s));
+        }
+    }
+    // 2. merge weights per (split, head)
+    float *weights = sm_red();  // [ns][64]
+    if (t < kHeads) {
+        int got = 1;
+        if (t == 0) got = wait_cluster_phase(&bars[kBarMl], 0, p) ? 1 : 0;
+        got = barrier_or(kBarIdHeads, kHeads, !got) ? 0 : 1;
+        if (got) (void)mbar_try_wait_cluster(&bars[kBarMl], 0);
+        float mv[kMaxClusterSplits], lv[kMaxClusterSplits];
+        bool bad = !got;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kMaxClusterSplits; ++s) {
+            mv[s] = -INFINITY;
+            lv[s] = 0.0f;
+            if (s < ns) {
+                mv[s] = (s == me) ? (ok ? sm_head_m()[t] : NAN) : __ldcg(ml + s * 128 + t);
+                lv[s] = (s == me) ? (ok ? sm_head_alpha()[t] : NAN) : __ldcg(ml + s * 128 + 64 + t);
+            }
+            bad = bad || isnan(mv[s]) || isnan(lv[s]);
+            if (lv[s] > 0.0f) mx = fmaxf(mx, mv[s]);
+        }
+        float sum = 0.0f;
+#pragma unroll
+        for (int s = 0; s < kMaxClusterSplits; ++s)
+            if (lv[s] > 0.0f) sum += exp2f(mv[s] - mx) * lv[s];
+        const float L = (sum > 0.0f) ? mx + log2f(sum) : -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kMaxClusterSplits; ++s)
+            if (s < ns) weights[s * kHeads + t] = bad ? NAN : (sum > 0.0f && lv[s] > 0.0f) ? exp2f(mv[s] - L) : 0.0f;
+        if (me == 0) p.lse[static_cast<size_t>(b) * kHeads + t] = bad ? NAN : (sum > 0.0f) ? L * 0.69314718055994531f
+                                                                                               : -INFINITY;
+    }
+    // the peers' receive buffers must be free before anything is sent (this barrier also
+    // publishes the weights)
+    const bool rx_ready = workers_wait_cluster(&bars[kBarRxReady], 0, p, t);
+    // 3. stream the units chunk by chunk as the last PV finishes them.  Each warp runs
+    //    its own loop: the unit of chunk c it covers depends only on c and on the peer
+    //    warps with the same index, which send chunk c before they wait for anything
+    //    of chunk c+1, so no warp waits on a warp that waits on it.
+    const int d = 32 * (w.q & 1) + w.lane;  // dim within the unit
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        const int u = 2 * c + (w.q >> 1);
+        const int o = u % ns;
+        const bool chunk_ok =
+            ok && n > 0 && warp_wait_phase(&bars[kBarKvFree + c], (n - 1) & 1, sm_abort(), p, w.lane);
+        float v[16];
+        if (chunk_ok) {
+            tmem_ld16(w.tmem + w.lane_base + 64 * c + 16 * w.hq, v);
+            tmem_wait_ld();
+        } else {
+            // no tile (O = 0, weight 0) or a failed wait (the result is invalid)
+#pragma unroll
+            for (int h = 0; h < 16; ++h) v[h] = (ok && n == 0) ? 0.0f : NAN;
+        }
+        if (o != me) {
+            // without rx_ready nothing is sent: the owner's wait runs out and it writes NaN
+            if (rx_ready) {
+                const int slot = (u / ns) * (ns - 1) + (me < o ? me : me - 1);
+                const uint32_t row = map_to_rank(g_smem + rx_base + slot * kUnitBytes + d * 256, o);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int g = (4 * w.hq + j) ^ (d & 7);
+                    st_cluster_v4(row + g * 16, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+                // one arrival per lane, releasing that lane's stores
+                mbar_arrive_remote(map_to_rank(&bars[kBarRx + u / ns], o));
+            }
+            continue;
+        }
+        int got = 1;
+        if (w.lane == 0) got = wait_cluster_phase(&bars[kBarRx + u / ns], 0, p) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (got) (void)mbar_try_wait_cluster(&bars[kBarRx + u / ns], 0);
+        float acc[16], wt[16];
+        load16(weights + me * kHeads + 16 * w.hq, wt);
+#pragma unroll
+        for (int h = 0; h < 16; ++h) acc[h] = (wt[h] != 0.0f) ? v[h] * wt[h] : 0.0f;  // NaN weights propagate
+        for (int s = 0; s < ns; ++s) {
+            if (s == me) continue;
+            const int slot = (u / ns) * (ns - 1) + (s < me ? s : s - 1);
+            const float *row = reinterpret_cast<const float *>(g_smem + rx_base + slot * kUnitBytes + d * 256);
+            load16(weights + s * kHeads + 16 * w.hq, wt);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 r = reinterpret_cast<const float4 *>(row)[(4 * w.hq + j) ^ (d & 7)];
+                const float rv[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ws = wt[4 * j + e];
+                    if (ws != 0.0f) acc[4 * j + e] += rv[e] * ws;
+                }
+            }
+        }
+        float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * w.hq) * kDim + 64 * u + d;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) dst[h * kDim] = got ? acc[h] : NAN;
+    }
+}
+
 // ------------------------------------------------------------------ the decode kernel
-// One CTA per (topk split, request), one 128-slot tile at a time, three warp roles
-// that hand work to each other through mbarriers:
-//   producers (8 warps): translate the slots of tile i+2 through the block table,
-//     keep the FP8 rows of tile i+1 in flight in registers, and dequantise tile i
-//     into the bf16 tile one K-block pair at a time, each pair as soon as the PV of
-//     tile i-1 has released it (so dequantisation overlaps the previous PV);
-//   MMA issue (lane 0 of softmax warp 0, between its softmax steps): once P^T of tile
-//     i is written, O^T += V^T.P_hi^T + V^T.P_lo^T (64 MMAs), committing each 128-dim
-//     chunk to the producers; then S^T = K.Q^T of tile i+1 (M=128 tokens, N=64
-//     heads) pair by pair as the producers publish them, into the other of two S^T
-//     buffers in tensor memory;
-//   softmax (8 warps; warp w reads TMEM lanes 32(w%4).. = tokens, columns for heads
-//     32(w/4)..): p = 2^(s*c - m) against the running max m, which is raised (with a
-//     rescale of O^T and of the per-thread sums) only when a score exceeds it by more
-//     than 2^8; P^T is written as bf16 hi + lo terms.
-// The epilogue reduces the per-thread sums and writes O/l and LSE, merging the splits of
-// a request inside its thread-block cluster when there are 2..4 of them.
+// One CTA per (topk split, request).  The 16 worker warps move one 128-slot tile at a
+// time through dequantisation and softmax while the rows of the next two tiles are in
+// flight; the control warp issues the MMAs (S^T of tile i as its dims chunks land,
+// PV of tile i once P^T is written, each PV chunk releasing that chunk of the tile
+// buffer to the next tile's dequantisation).
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_q) {
-    extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int split = blockIdx.x;
     const int b = blockIdx.y;
 
-    if (smem_addr(smem) & 1023u) {
+    // The dynamic shared memory base is the same for every CTA of the launch, so this
+    // exit is uniform: no CTA of a cluster can be left waiting for a peer that took it.
+    if (smem_addr(g_smem) & 1023u) {
         if (tid == 0) atomicOr(p.err, SMLA_FLAG_SMEM);
         return;
     }
-    uint8_t *sQ = smem + kSmemQ;
-    uint8_t *sKV = smem + kSmemKV;
-    int *codes = reinterpret_cast<int *>(smem + kSmemCodes);
-    uint32_t *mask = reinterpret_cast<uint32_t *>(smem + kSmemMask);
-    float *head_m = reinterpret_cast<float *>(smem + kSmemHeadM);
-    float *head_alpha = reinterpret_cast<float *>(smem + kSmemHeadAlpha);
-    float *red = reinterpret_cast<float *>(smem + kSmemRed);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBars);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmemTmemSlot);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmemAbort);
+    uint64_t *bars = sm_bars();
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(g_smem + kSmemTmemSlot);
+    int *codes = sm_codes();
+    uint32_t *mask = sm_mask();
+    float *head_m = sm_head_m();
 
     const int num_tiles = (p.topk + kTile - 1) / kTile;
     const int t_begin = split * p.tiles_per_split;
@@ -558,269 +928,98 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int seq_len = __ldg(p.seq_lens + b);
     const int32_t *bt_row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
     const int32_t *idx_row = p.topk_idx + static_cast<size_t>(b) * p.topk;
+    const int ns = p.nsplit;
 
     // ---- setup
-    if (warp == 0) {
+    Translator tr;
+    if (warp == kCtlWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
         if (lane == 0) {
             mbar_init(&bars[kBarQ], 1);
             for (int c = 0; c < 4; ++c) {
-                mbar_init(&bars[kBarKvFull + c], kProducerWarps);
+                mbar_init(&bars[kBarKvFull + c], kWorkerWarps);
                 mbar_init(&bars[kBarKvFree + c], 1);
+                mbar_init(&bars[kBarRx + c], p.cluster_merge ? (ns - 1) * 8 * 32 : 1);  // 8 warps per peer
             }
             mbar_init(&bars[kBarSFull], 1);
             mbar_init(&bars[kBarSFull + 1], 1);
-            mbar_init(&bars[kBarPFull], kSoftmaxWarps);
+            mbar_init(&bars[kBarPFull], kWorkerWarps);
             mbar_init(&bars[kBarDrain], 1);
             mbar_init(&bars[kBarSpare], 1);
-            mbar_init(&bars[kBarXch], 1);
+            mbar_init(&bars[kBarMl], (p.cluster_merge && ns > 2) ? ns - 1 : 1);
+            mbar_init(&bars[kBarRxReady], p.cluster_merge ? ns - 1 : 1);
+            // two splits: the peer's row of 64 log-sum-exps arrives as 256 transaction bytes
+            if (p.cluster_merge && ns == 2) mbar_arrive_expect_tx(&bars[kBarMl], kHeads * 4);
             fence_barrier_init();
-            *abort_flag = 0;
+            *sm_abort() = 0;
             mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
 #pragma unroll
-            for (int kb = 0; kb < 8; ++kb) tma_load_2d(sQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
+            for (int kb = 0; kb < 8; ++kb) tma_load_2d(g_smem + kSmemQ + kb * 8192, &tmap_q, 64 * kb, kHeads * b, &bars[kBarQ]);
         }
-    } else if (warp >= kSoftmaxWarps) {
-        // index translation of tiles 0 and 1 (producer thread pt: tile pt/128, slot pt%128)
-        const int pt = tid - kSoftmaxThreads;
-        const int ti = pt >> 7;
-        const int slot = (t_begin + ti) * kTile + (pt & (kTile - 1));
+    } else if (tid < 2 * kTile) {
+        // index translation of tiles 0 and 1 (worker t: tile t / 128, slot t % 128)
+        const int ti = tid >> 7;
+        const int s = slot_index(p, t_begin, ti, tid & (kTile - 1));
         int code = -1;
-        if (ti < n && slot < p.topk)
-            code = translate_slot(bt_row, p.max_blocks, seq_len, p.num_pages, __ldg(idx_row + slot), p.err);
-        codes[pt] = code;
+        if (ti < n && s < p.topk)
+            code = translate_slot(bt_row, p.max_blocks, seq_len, p.num_pages, __ldg(idx_row + s), p.err);
+        codes[tid] = code;
         const uint32_t bits = __ballot_sync(0xffffffffu, code >= 0);
-        if (lane == 0) mask[ti * 4 + ((pt >> 5) & 3)] = bits;
+        if (lane == 0) mask[ti * 4 + ((tid >> 5) & 3)] = bits;
+        if (tid < kTile && n > 2) {
+            const int s2 = slot_index(p, t_begin, 2, tid);
+            tr.idx_a = (s2 < p.topk) ? __ldg(idx_row + s2) : -1;
+        }
     }
     if (tid < kHeads) head_m[tid] = -INFINITY;
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
-    const float c = p.scale_log2;
-
-    if (warp < kSoftmaxWarps) {
-        // ================================================================ softmax (+ MMA issue)
-        const int q = warp & 3;
-        const int hh = warp >> 2;
-        const int r = 32 * q + lane;  // token lane of S^T
-        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-        const uint32_t phi_s = smem_addr(smem + kSmemPhi);
-        const uint32_t plo_s = smem_addr(smem + kSmemPlo);
-        const bool issuer = (tid == 0);
-        MmaIssuer mma(smem, tmem, p, bars, abort_flag);
-        if (issuer && n > 0) mma.qk(0);
-        __syncwarp();
-        bool failed = false;
-        for (int i = 0; i < n; ++i) {
-            const int sb = i & 1;
-            const uint32_t s_cols = tmem + lane_base + kTmemS + 64 * sb + 32 * hh;
-            const uint32_t l_cols = tmem + lane_base + kTmemL + 32 * hh;
-            const bool ok = warp_wait_phase(&bars[kBarSFull + sb], (i >> 1) & 1, abort_flag, p, lane);
-            if (barrier_or(kBarIdSoftmax, kSoftmaxThreads, !ok)) {
-                failed = true;
-                break;
-            }
-            tc_fence_after_sync();
-            const bool valid = (mask[(i & 3) * 4 + q] >> lane) & 1u;
-            // does any score exceed its head's running max by more than the threshold?
-            bool over = false;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float x[16];
-                tmem_ld16(s_cols + 16 * half, x);
-                tmem_wait_ld();
-                float m[16];
-                load16(head_m + 32 * hh + 16 * half, m);
-#pragma unroll
-                for (int h = 0; h < 16; ++h) over |= valid && (x[h] * c - m[h]) > kRescaleThreshold;
-            }
-            if (barrier_or(kBarIdSoftmax, kSoftmaxThreads, over)) {
-                // raise each head's running max to max(m, tile max); rescale what was accumulated
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float x[16];
-                    tmem_ld16(s_cols + 16 * half, x);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) x[h] = valid ? x[h] * c : -INFINITY;
-                    const float tmax = warp_transpose_reduce<true, 16>(x, lane);
-                    if ((lane & 1) == 0) red[q * 64 + 32 * hh + 16 * half + (lane >> 1)] = tmax;
-                }
-                named_barrier_sync(kBarIdSoftmax, kSoftmaxThreads);
-                if (tid < kHeads) {
-                    const float tm = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
-                    const float mo = head_m[tid];
-                    const float mn = fmaxf(mo, tm);
-                    head_alpha[tid] = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
-                    head_m[tid] = mn;
-                }
-                named_barrier_sync(kBarIdSoftmax, kSoftmaxThreads);
-                if (i > 0) {
-                    // the PV of tile i-1 is complete (the S^T commit of tile i covers it): rescale
-                    // the 4 O^T chunks and the sums, 16 heads at a time
-#pragma unroll 1
-                    for (int part = 0; part < 10; ++part) {
-                        const int h0 = 16 * (part & 1);
-                        const uint32_t col = (part < 8 ? tmem + lane_base + 64 * (part >> 1) + 32 * hh : l_cols) + h0;
-                        float o[16], al[16];
-                        tmem_ld16(col, o);
-                        load16(head_alpha + 32 * hh + h0, al);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int h = 0; h < 16; ++h) o[h] *= al[h];
-                        tmem_st16(col, o);
-                    }
-                }
-            }
-            // p = 2^(s c - m): add to the sums, write P^T row r as bf16 hi + lo
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float x[16], l[16];
-                tmem_ld16(s_cols + 16 * half, x);
-                if (i > 0) tmem_ld16(l_cols + 16 * half, l);
-                tmem_wait_ld();
-                float m[16];
-                load16(head_m + 32 * hh + 16 * half, m);
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                    x[h] = valid ? fast_exp2(x[h] * c - m[h]) : 0.0f;
-                    l[h] = (i > 0) ? l[h] + x[h] : x[h];
-                }
-                tmem_st16(l_cols + 16 * half, l);
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float a0 = x[8 * j + 2 * e], a1 = x[8 * j + 2 * e + 1];
-                        hw[e] = pack_bf16x2(a0, a1);
-                        lw[e] = pack_bf16x2(a0 - __uint_as_float(hw[e] << 16), a1 - __uint_as_float(hw[e] & 0xFFFF0000u));
-                    }
-                    const uint32_t off = r * 128 + (((4 * hh + 2 * half + j) ^ (r & 7)) << 4);
-                    sts_v4(phi_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-                    sts_v4(plo_s + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
-                }
-            }
-            fence_proxy_async_smem();
-            tmem_wait_st();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kBarPFull]);
-            // warp 0's lane 0 issues PV of this tile and QK of the next one while the other
-            // softmax warps wait for that S^T
-            if (issuer && mma.pv(i) && i + 1 < n) mma.qk(i + 1);
-            __syncwarp();
-        }
-        // the last PV is complete before the epilogue reads O^T
-        if (!failed && n > 0) {
-            const bool ok = warp_wait_phase(&bars[kBarKvFree + 3], (n - 1) & 1, abort_flag, p, lane);
-            (void)barrier_or(kBarIdSoftmax, kSoftmaxThreads, !ok);
-        }
-        // every MMA issued must be complete before tensor memory is released
-        if (issuer) mma.drain();
-        __syncwarp();
-        tc_fence_after_sync();
-        // per-head sums over this warp's 32 token lanes
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            float l[16];
-            if (n > 0 && !failed) {
-                tmem_ld16(tmem + lane_base + kTmemL + 32 * hh + 16 * half, l);
-                tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int h = 0; h < 16; ++h) l[h] = 0.0f;
-            }
-            const float ls = warp_transpose_reduce<false, 16>(l, lane);
-            if ((lane & 1) == 0) red[q * 64 + 32 * hh + 16 * half + (lane >> 1)] = ls;
-        }
-    } else {
-        // ================================================================ producers
-        const int pt = tid - kSoftmaxThreads;
-        const uint32_t kv_s = smem_addr(sKV);
-        TileRegs tr;
-        if (n > 0) load_tile(pt, codes, p.cache, tr);
-        for (int i = 0; i < n; ++i) {
-            const int buf = i & 1;
-            // translation of tile i+2, first step: its topk indices
-            const int slot2 = (t_begin + i + 2) * kTile + pt;
-            int idx_next = -1;
-            if (pt < kTile && i + 2 < n && slot2 < p.topk) idx_next = __ldg(idx_row + slot2);
-            bool ok = produce_tile(i, pt, lane, kv_s, bars, abort_flag, p, tr);
-            // second step: the block-table entries
-            int page_next = -1;
-            const bool in_range = idx_next >= 0 && idx_next < seq_len && (idx_next >> 8) < p.max_blocks;
-            if (in_range) page_next = __ldg(bt_row + (idx_next >> 8));
-            // the rows of tile i+1 go in flight
-            if (ok && i + 1 < n) load_tile(pt, codes + (buf ^ 1) * kTile, p.cache, tr);
-            // tile i+2's codes replace tile i's (the loads above read the other buffer)
-            if (pt < kTile && i + 2 < n) {
-                int code = -1;
-                if (in_range) {
-                    if (page_next < 0 || static_cast<long long>(page_next) >= p.num_pages)
-                        atomicOr(p.err, SMLA_FLAG_BAD_PAGE);
-                    else
-                        code = page_next * kPageTokens + (idx_next & (kPageTokens - 1));
-                }
-                codes[buf * kTile + pt] = code;
-                const uint32_t bits = __ballot_sync(0xffffffffu, code >= 0);
-                if (lane == 0) mask[((i + 2) & 3) * 4 + (pt >> 5)] = bits;
-            }
-            if (barrier_or(kBarIdProducer, kProducerThreads, !ok)) break;
-        }
+    if (p.cluster_merge && ns == 2) {
+        // two splits add their weighted partials into the output: each CTA zeroes 32 heads of
+        // out[b] now; the barriers below order these stores before either CTA's additions
+        float4 *z = reinterpret_cast<float4 *>(p.out + (static_cast<size_t>(b) * kHeads + 32 * split) * kDim);
+        for (int k = tid; k < 32 * kDim / 4; k += kThreads) z[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    const bool ok = !*abort_flag;
+    if (p.cluster_merge) cluster_arrive();  // peers may address this CTA's mbarriers from now on
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
 
-    // ---- epilogue: per-head sums (red holds them per TMEM quadrant), then O/l or the cluster merge
-    float *l_head = head_alpha;
-    if (tid < kHeads) l_head[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
+    if (warp == kCtlWarp) {
+        // ================================================================ MMA issue
+        if (lane == 0 && n > 0) mma_issue_loop(tmem, p, n);
+        __syncwarp();
+        if (p.cluster_merge) cluster_wait();
+    } else {
+        // ================================================================ workers
+        Worker w{p, tmem, tid, warp, lane, warp & 3, warp >> 2, static_cast<uint32_t>(32 * (warp & 3)) << 16};
+        Slot slot;
+        if (n > 0) load_slot(tid, codes, p.cache, slot);
+        // tile 1's rows head for L2 right behind tile 0's (its register loads come later)
+        if (tid >= kTile && tid < 2 * kTile && codes[tid] >= 0) prefetch_token_l2(p.cache, codes[tid]);
+        for (int i = 0; i < n && ok; ++i) ok = worker_step(w, i, n, t_begin, seq_len, bt_row, idx_row, tr, slot);
+        ok = ok && !*sm_abort();
+        ok = !barrier_or(kBarIdWorkers, kWorkers, !ok);
+        w.reduce_sums(ok && n > 0);
+        if (p.cluster_merge) {
+            cluster_wait();  // every peer has initialised its mbarriers (and zeroed its part of out)
+            if (ns == 2)
+                epilogue_pair(w, b, n, ok);
+            else
+                epilogue_cluster(w, b, n, ok);
+        } else {
+            epilogue_direct(w, b, split, n, ok);
+        }
+    }
+    tc_fence_before_sync();
     __syncthreads();
     if (p.cluster_merge) {
-        cluster_epilogue(p, b, ok, n, tid, warp, lane, tmem, smem, &bars[kBarXch], head_m, l_head, red);
-    } else if (ok) {
-        if (tid < kHeads) {
-            const float l = l_head[tid];
-            const float val = (l > 0.0f) ? (head_m[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-            if (p.nsplit == 1)
-                p.lse[static_cast<size_t>(b) * kHeads + tid] = val;
-            else
-                p.part_lse[(static_cast<size_t>(b) * kHeads + tid) * p.nsplit + split] = val;
-        }
-        if (tid < kHeads) {
-            const float l = l_head[tid];
-            red[tid] = (l > 0.0f) ? 1.0f / l : 0.0f;  // 1/l per head
-        }
-        __syncthreads();
-        if (warp < kSoftmaxWarps) {
-            const int q = warp & 3;
-            const int hh = warp >> 2;
-            const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-            // the nsplit > 1 partials are [b][head][split][dim]
-            const size_t head_stride = static_cast<size_t>(p.nsplit) * kDim;
-            float *base = (p.nsplit == 1) ? p.out + static_cast<size_t>(b) * kHeads * kDim
-                                          : p.part_o + static_cast<size_t>(b) * kHeads * head_stride + split * kDim;
-#pragma unroll 1
-            for (int part = 0; part < 8; ++part) {  // 4 chunks x 2 halves of 16 heads
-                const int mc = part >> 1, h0 = 32 * hh + 16 * (part & 1);
-                float o[16];
-                if (n > 0) {
-                    tmem_ld16(tmem + lane_base + 64 * mc + h0, o);
-                    tmem_wait_ld();
-                }
-                float *dst = base + static_cast<size_t>(h0) * head_stride + 128 * mc + 32 * q + lane;
-#pragma unroll
-                for (int h = 0; h < 16; ++h) dst[h * head_stride] = (n > 0) ? o[h] * red[h0 + h] : 0.0f;
-            }
-        }
+        // no CTA leaves while a peer may still write into its shared memory
+        cluster_arrive();
+        cluster_wait();
     }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
+    if (warp == kCtlWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -834,8 +1033,18 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
     const int tid = threadIdx.x;
     const float *L = part_lse + bh * nsplit;
     float lmax = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) lmax = fmaxf(lmax, __ldg(L + s));
+    bool invalid = false;  // a NaN partial LSE marks a split whose CTA aborted
+    for (int s = 0; s < nsplit; ++s) {
+        const float ls = __ldg(L + s);
+        invalid = invalid || isnan(ls);
+        lmax = fmaxf(lmax, ls);
+    }
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (invalid) {
+        reinterpret_cast<float4 *>(out + bh * kDim)[tid] = make_float4(NAN, NAN, NAN, NAN);
+        if (tid == 0) lse[bh] = NAN;
+        return;
+    }
     if (lmax == -INFINITY) {
         reinterpret_cast<float4 *>(out + bh * kDim)[tid] = acc;
         if (tid == 0) lse[bh] = -INFINITY;
@@ -1005,23 +1214,20 @@ bool sizes_ok(int B, int H, int topk) {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Up to this many splits of a request merge inside a thread-block cluster (exchanging
-// through the workspace, ordered by the cluster barrier); beyond it they go through
-// normalised global partials and the merge kernel.
-constexpr int kMaxClusterSplits = 4;
-
+// Up to smla::kMaxClusterSplits splits of a request merge inside a thread-block cluster
+// (partial outputs travel through distributed shared memory); beyond it they go
+// through normalised global partials and the merge kernel.
+//
 // Workspace after the header: nsplit == 1: nothing.  2..4 (cluster merge): the
-// (m, l) rows [B][nsplit][128] f32, then the exchanged O^T chunks
-// [B][4][nsplit-1][64][128] f32.  Above 4: part_lse [B][64][nsplit] f32, then
-// part_o [B][64][nsplit][512] f32.
+// per-split (m, l) rows [B][nsplit][128] f32.  Above 4: part_lse [B][64][nsplit]
+// f32, then part_o [B][64][nsplit][512] f32.
 size_t workspace_for(int B, int topk, int nsplit) {
     size_t bytes = SMLA_WORKSPACE_HEADER;
-    if (nsplit > kMaxClusterSplits) {
+    if (nsplit > smla::kMaxClusterSplits) {
         const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
         bytes += round256(rows * sizeof(float)) + rows * SMLA_DIM * sizeof(float);
     } else if (nsplit > 1) {
-        bytes += round256(static_cast<size_t>(B) * nsplit * 128 * sizeof(float)) +
-                 static_cast<size_t>(B) * 4 * (nsplit - 1) * 128 * SMLA_HEADS * sizeof(float);
+        bytes += round256(static_cast<size_t>(B) * nsplit * 128 * sizeof(float));
     }
     (void)topk;
     return bytes;
@@ -1096,8 +1302,8 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     p.lse = lse;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.err = reinterpret_cast<uint32_t *>(ws);
-    const size_t rows = (nsplit > kMaxClusterSplits) ? static_cast<size_t>(B) * SMLA_HEADS * nsplit
-                                                             : static_cast<size_t>(B) * nsplit * 128;
+    const size_t rows = (nsplit > smla::kMaxClusterSplits) ? static_cast<size_t>(B) * SMLA_HEADS * nsplit
+                                                           : static_cast<size_t>(B) * nsplit * 128;
     p.part_lse = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER);
     p.part_o = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER + round256(rows * sizeof(float)));
     p.num_pages = num_pages;
@@ -1115,7 +1321,7 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     (void)cudaGetLastError();
-    p.cluster_merge = (nsplit > 1 && nsplit <= kMaxClusterSplits) ? 1 : 0;
+    p.cluster_merge = (nsplit > 1 && nsplit <= smla::kMaxClusterSplits) ? 1 : 0;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(nsplit, B);
     cfg.blockDim = dim3(smla::kThreads);

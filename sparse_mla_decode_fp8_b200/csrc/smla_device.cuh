@@ -32,19 +32,29 @@ static_assert(kPageBytes % 128 == 0, "pages must stay 128-byte aligned");
 static_assert(kPageBytes == kPageTokens * (kRowBytes + kScaleRowBytes), "page size");
 static_assert(kScaleBlockOffset == kPageTokens * kRowBytes, "scale block follows the rows");
 
-// Token code = page * 256 + slot for a valid topk slot, else -1.  A block-table
-// entry outside [0, num_pages) is masked and reported in the error word.
-__device__ __forceinline__ int translate_slot(const int32_t *bt_row, int max_blocks, int seq_len,
-                                              long long num_pages, int idx, uint32_t *err) {
-    if (idx < 0 || idx >= seq_len) return -1;
-    const int blk = idx >> 8;
-    if (blk >= max_blocks) return -1;
-    const int page = __ldg(bt_row + blk);
+// Index translation in two steps, so a caller can put the block-table load between
+// them (the decode kernel keeps that load in flight while it computes).
+//   1. slot_in_range: 0 <= idx < seq_len and idx / 256 < max_blocks; only then is
+//      block_table[b][idx / 256] read.
+//   2. slot_code: token code = page * 256 + idx % 256, or -1 (and the error bit)
+//      for a block-table entry outside [0, num_pages).
+__device__ __forceinline__ bool slot_in_range(int idx, int seq_len, int max_blocks) {
+    return idx >= 0 && idx < seq_len && (idx >> 8) < max_blocks;
+}
+__device__ __forceinline__ int slot_code(int idx, int page, long long num_pages, uint32_t *err) {
     if (page < 0 || static_cast<long long>(page) >= num_pages) {
         atomicOr(err, SMLA_FLAG_BAD_PAGE);
         return -1;
     }
     return page * kPageTokens + (idx & (kPageTokens - 1));
+}
+
+// Token code = page * 256 + slot for a valid topk slot, else -1.  A block-table
+// entry outside [0, num_pages) is masked and reported in the error word.
+__device__ __forceinline__ int translate_slot(const int32_t *bt_row, int max_blocks, int seq_len,
+                                              long long num_pages, int idx, uint32_t *err) {
+    if (!slot_in_range(idx, seq_len, max_blocks)) return -1;
+    return slot_code(idx, __ldg(bt_row + (idx >> 8)), num_pages, err);
 }
 
 __device__ __forceinline__ const uint8_t *token_row(const uint8_t *cache, int code) {
