@@ -654,11 +654,12 @@ __device__ __forceinline__ bool worker_step(Worker &w, int i, int n, int t_begin
 
 // ------------------------------------------------------------------ epilogues
 // Writes dims chunk c of this CTA's O^T, each head h scaled by scale[h] (16 heads 16hq..,
-// in registers), to dst + h * head_stride + 128c + dim with 16-byte accesses: the warp
-// stages its 16 heads x 32 dims through the (dead) Q buffer as [head][dim] rows, then
-// every lane writes 4 consecutive dims of a head (plain stores, or atomic adds into an
-// output the splits share).  What is written: kChunkTmem the scaled O^T, kChunkZero zeros
-// (no tile, or weight 0), kChunkNan NaN (a failed wait: the result is invalid).
+// in registers), to dst + h * head_stride + 128c + dim.  Lane l of warp (q, hq) holds dim
+// 32q + l of its 16 heads, so each store or atomic add of a head covers 32 consecutive
+// floats per warp (128 bytes, coalesced) without staging through shared memory, whose
+// bandwidth the tensor core is using meanwhile.  What is written: kChunkTmem the scaled
+// O^T, kChunkZero zeros (no tile, or weight 0), kChunkNan NaN (a failed wait: the result
+// is invalid).
 enum ChunkSource : int { kChunkNan = 0, kChunkZero = 1, kChunkTmem = 2 };
 __device__ __forceinline__ void write_chunk(const Worker &w, int c, const float (&scale)[16], float *dst,
                                             size_t head_stride, int source, bool add) {
@@ -667,30 +668,17 @@ __device__ __forceinline__ void write_chunk(const Worker &w, int c, const float 
         tmem_ld16(w.tmem + w.lane_base + 64 * c + 16 * w.hq, v);
         tmem_wait_ld();
     }
-    float *stage = reinterpret_cast<float *>(g_smem + kSmemQ);  // [64 heads][128 dims] f32
+    float *o = dst + static_cast<size_t>(16 * w.hq) * head_stride + 128 * c + 32 * w.q + w.lane;
 #pragma unroll
-    for (int h = 0; h < 16; ++h)
-        stage[(16 * w.hq + h) * 128 + 32 * w.q + w.lane] =
-            (source == kChunkTmem) ? v[h] * scale[h] : (source == kChunkZero) ? 0.0f : NAN;
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int h = 16 * w.hq + 4 * k + (w.lane >> 3);
-        const int d = 32 * w.q + 4 * (w.lane & 7);
-        const float4 x = *reinterpret_cast<const float4 *>(stage + h * 128 + d);
-        float *o = dst + static_cast<size_t>(h) * head_stride + 128 * c + d;
+    for (int h = 0; h < 16; ++h) {
+        const float x = (source == kChunkTmem) ? v[h] * scale[h] : (source == kChunkZero) ? 0.0f : NAN;
         if (add)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o), "f"(x.x), "f"(x.y), "f"(x.z),
-                         "f"(x.w)
-                         : "memory");
+            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(o + h * head_stride), "f"(x) : "memory");
         else
-            *reinterpret_cast<float4 *>(o) = x;
+            o[h * head_stride] = x;
     }
-    __syncwarp();
 }
 
-// nsplit = 1: O = O^T / l and LSE; nsplit > 4: normalised partials for the merge
-// kernel.  A CTA that aborted writes NaN (its rows are then visibly invalid).
 __device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int n, bool ok) {
     const DecodeParams &p = w.p;
     if (n > 0) ok = workers_wait(&sm_bars()[kBarKvFree + 3], (n - 1) & 1, p, w.t, ok);
@@ -753,8 +741,11 @@ __device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) 
     float sc[16];
     load16(scale + 16 * w.hq, sc);
     float *base = p.out + static_cast<size_t>(b) * kHeads * kDim;
+    // the two CTAs add into the same output, in chunk orders two chunks apart, so that
+    // their atomic adds do not meet on the same lines at the same time
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int k = 0; k < 4; ++k) {
+        const int c = (k + 2 * me) & 3;
         const bool chunk_ok = workers_wait(&bars[kBarKvFree + c], (n - 1) & 1, p, t, ok && n > 0);
         // a split without tiles adds zeros; a failed wait NaN
         const int source = chunk_ok ? kChunkTmem : (ok && n == 0) ? kChunkZero : kChunkNan;
