@@ -92,13 +92,20 @@ constexpr int kSmemBytes = kSmemAbort + 4;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-block shared memory limit");
 static_assert(kSmemBars % 8 == 0, "mbarriers need 8-byte alignment");
 
-// Tensor memory: O^T [0,256) (4 chunks of 128 dims x 64 heads), S^T buffers at 256 and 320,
-// per-lane running sums L at 384 (lane = token row of the tile, column = head).
+// Tensor memory (lane = dim of an O^T chunk, or token row of S^T and L; column = head):
+//   [0, 256)   O^T dims chunks 0 and 1, 128 columns each: V^T.P_hi^T | V^T.P_lo^T
+//              (one N = 128 MMA per step reads V^T once for both terms)
+//   [256, 384) O^T dims chunks 2 and 3, 64 columns each: both terms accumulate in place
+//   [384, 448) S^T of the current tile (dead before the next tile's QK^T is issued:
+//              that waits for the dequantisation, which waits for this tile's PV)
+//   [448, 512) per-lane running sums L
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 256;
-constexpr uint32_t kTmemL = 384;
+constexpr uint32_t kTmemO2 = 256;
+constexpr uint32_t kTmemS = 384;
+constexpr uint32_t kTmemL = 448;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 64, true, true);
+constexpr uint32_t kIdescPV2 = idesc_bf16(128, 128, true, true);
 // log2 units: the running max m of a head is raised (and O^T, the sums rescaled) only when a
 // score exceeds it by more than this, so p = 2^(s - m) stays below 2^64.  P_hi + P_lo keep
 // their relative precision at any magnitude, and fp32 sums of p x |v| over at most 2^16 slots
@@ -415,7 +422,7 @@ __device__ __forceinline__ void issue_qk_chunk(uint32_t d, uint32_t a_lo, uint32
 }
 
 // O^T chunk += V^T.P_hi^T + V^T.P_lo^T over the tile's 128 tokens: 8 steps of 16 tokens
-// (2 KB apart in the MN-major V^T and P^T).
+// (2 KB apart in the MN-major V^T and P^T), two N = 64 MMAs per step.
 __device__ __forceinline__ void issue_pv_chunk(uint32_t d, uint32_t a_lo, uint32_t bh_lo, uint32_t bl_lo,
                                                bool accumulate) {
     if (accumulate)
@@ -431,7 +438,21 @@ __device__ __forceinline__ void issue_pv_chunk(uint32_t d, uint32_t a_lo, uint32
     }
 }
 
-// For each tile i: S^T = K.Q^T into buffer i&1 chunk by chunk as the workers publish the
+// [O^T_hi | O^T_lo] chunk += V^T.[P_hi | P_lo]^T: one N = 128 MMA per step of 16 tokens,
+// whose B operand is the two P^T arrays as two 64-column MN blocks 16 KB apart.
+__device__ __forceinline__ void issue_pv_wide(uint32_t d, uint32_t a_lo, uint32_t b_lo, bool accumulate) {
+    if (accumulate)
+        mma_bf16_ss_acc(d, desc_from(a_lo, kDescHi), desc_from(b_lo, kDescHi), kIdescPV2);
+    else
+        mma_bf16_ss(d, desc_from(a_lo, kDescHi), desc_from(b_lo, kDescHi), kIdescPV2, 0u);
+#pragma unroll
+    for (int ks = 1; ks < 8; ++ks) {
+        const uint32_t o = ks * (2048 >> 4);
+        mma_bf16_ss_acc(d, desc_from(a_lo + o, kDescHi), desc_from(b_lo + o, kDescHi), kIdescPV2);
+    }
+}
+
+// For each tile i: S^T = K.Q^T chunk by chunk as the workers publish the
 // tile's dims chunks, then, once every worker has written P^T, O^T += V^T.P^T with a
 // commit per 128-dim chunk (freeing that chunk of the tile buffer; in the last tile it
 // makes that chunk of O^T final).
@@ -443,9 +464,10 @@ __device__ __forceinline__ void mma_issue_loop(uint32_t tmem, const DecodeParams
     const uint32_t pv_a = desc_lo(kv, kTile * 128);
     const uint32_t pv_bh = desc_lo(smem_addr(g_smem + kSmemPhi), 8192);
     const uint32_t pv_bl = desc_lo(smem_addr(g_smem + kSmemPlo), 8192);
+    const uint32_t pv_b2 = desc_lo(smem_addr(g_smem + kSmemPhi), kSmemPlo - kSmemPhi);
     bool ok = true, spare_used = false;
     for (int i = 0; i < n && ok; ++i) {
-        const uint32_t s_col = tmem + kTmemS + 64 * (i & 1);
+        const uint32_t s_col = tmem + kTmemS;
 #pragma unroll 1
         for (int cp = 0; cp < 4 && ok; ++cp) {
             ok = (i > 0 || cp > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
@@ -462,8 +484,13 @@ __device__ __forceinline__ void mma_issue_loop(uint32_t tmem, const DecodeParams
         if (!ok) break;
         tc_fence_after_sync();
 #pragma unroll 1
-        for (int mc = 0; mc < 4; ++mc) {
-            issue_pv_chunk(tmem + 64 * mc, pv_a + mc * 2 * ((kTile * 128) >> 4), pv_bh, pv_bl, i > 0);
+        for (int mc = 0; mc < 2; ++mc) {
+            issue_pv_wide(tmem + 128 * mc, pv_a + mc * 2 * ((kTile * 128) >> 4), pv_b2, i > 0);
+            mma_commit(&bars[kBarKvFree + mc]);
+        }
+#pragma unroll 1
+        for (int mc = 2; mc < 4; ++mc) {
+            issue_pv_chunk(tmem + kTmemO2 + 64 * (mc - 2), pv_a + mc * 2 * ((kTile * 128) >> 4), pv_bh, pv_bl, i > 0);
             mma_commit(&bars[kBarKvFree + mc]);
         }
     }
@@ -492,7 +519,7 @@ struct Worker {
         tc_fence_after_sync();
         const float c = p.scale_log2;
         const bool valid = (sm_mask()[(i & 3) * 4 + q] >> lane) & 1u;
-        const uint32_t s_col = tmem + lane_base + kTmemS + 64 * sb + 16 * hq;
+        const uint32_t s_col = tmem + lane_base + kTmemS + 16 * hq;
         const float4 *hm4 = reinterpret_cast<const float4 *>(sm_head_m() + 16 * hq);
         // does any score exceed its head's running max by more than the threshold?
         bool over = false;
@@ -570,7 +597,7 @@ struct Worker {
         named_barrier_sync(kBarIdWorkers, kWorkers);
         if (i == 0) return;  // nothing accumulated yet
         // the PV of tile i-1 is complete (the S^T commit of tile i covers it): rescale the
-        // 4 O^T chunks and the sums, unless none of this warp's 16 heads moved
+        // six 64-column groups of O^T and the sums, unless none of this warp's 16 heads moved
         float al[16];
         load16(sm_head_alpha() + 16 * hq, al);
         bool moved = false;
@@ -578,8 +605,8 @@ struct Worker {
         for (int h = 0; h < 16; ++h) moved |= al[h] != 1.0f;
         if (!moved) return;
 #pragma unroll 1
-        for (int mc = 0; mc < 5; ++mc) {
-            const uint32_t col = tmem + lane_base + (mc < 4 ? 64 * mc : kTmemL) + 16 * hq;
+        for (int mc = 0; mc < 7; ++mc) {
+            const uint32_t col = tmem + lane_base + (mc < 6 ? 64 * mc : kTmemL) + 16 * hq;
             float o[16];
             tmem_ld16(col, o);
             tmem_wait_ld();
@@ -653,6 +680,22 @@ __device__ __forceinline__ bool worker_step(Worker &w, int i, int n, int t_begin
 }
 
 // ------------------------------------------------------------------ epilogues
+// This lane's dim of O^T dims chunk c for the 16 heads 16hq..: chunks 0 and 1 keep the
+// P_hi and P_lo products in separate halves, added here.
+__device__ __forceinline__ void load_o16(uint32_t lane_addr, int c, int hq, float (&v)[16]) {
+    if (c < 2) {
+        float lo[16];
+        tmem_ld16(lane_addr + 128 * c + 16 * hq, v);
+        tmem_ld16(lane_addr + 128 * c + 64 + 16 * hq, lo);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 16; ++h) v[h] += lo[h];
+    } else {
+        tmem_ld16(lane_addr + kTmemO2 + 64 * (c - 2) + 16 * hq, v);
+        tmem_wait_ld();
+    }
+}
+
 // Writes dims chunk c of this CTA's O^T, each head h scaled by scale[h] (16 heads 16hq..,
 // in registers), to dst + h * head_stride + 128c + dim.  Lane l of warp (q, hq) holds dim
 // 32q + l of its 16 heads, so each store or atomic add of a head covers 32 consecutive
@@ -664,10 +707,7 @@ enum ChunkSource : int { kChunkNan = 0, kChunkZero = 1, kChunkTmem = 2 };
 __device__ __forceinline__ void write_chunk(const Worker &w, int c, const float (&scale)[16], float *dst,
                                             size_t head_stride, int source, bool add) {
     float v[16];
-    if (source == kChunkTmem) {
-        tmem_ld16(w.tmem + w.lane_base + 64 * c + 16 * w.hq, v);
-        tmem_wait_ld();
-    }
+    if (source == kChunkTmem) load_o16(w.tmem + w.lane_base, c, w.hq, v);
     float *o = dst + static_cast<size_t>(16 * w.hq) * head_stride + 128 * c + 32 * w.q + w.lane;
 #pragma unroll
     for (int h = 0; h < 16; ++h) {
@@ -835,8 +875,7 @@ __device__ __forceinline__ void epilogue_cluster(Worker &w, int b, int n, bool o
             ok && n > 0 && warp_wait_phase(&bars[kBarKvFree + c], (n - 1) & 1, sm_abort(), p, w.lane);
         float v[16];
         if (chunk_ok) {
-            tmem_ld16(w.tmem + w.lane_base + 64 * c + 16 * w.hq, v);
-            tmem_wait_ld();
+            load_o16(w.tmem + w.lane_base, c, w.hq, v);
         } else {
             // no tile (O = 0, weight 0) or a failed wait (the result is invalid)
 #pragma unroll
