@@ -251,9 +251,9 @@ __device__ __noinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parity, 
 // the barrier (every worker calls these with the same arguments).  Returns false if
 // the wait failed or was skipped.
 __device__ __forceinline__ bool workers_wait(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
-                                             bool enabled = true) {
+                                             bool enabled = true, uint32_t backoff_ns = kWorkerBackoffNs) {
     bool ok = enabled;
-    if (t == kWaiter && enabled) ok = wait_phase(bar, parity, sm_abort(), p, kWorkerBackoffNs);
+    if (t == kWaiter && enabled) ok = wait_phase(bar, parity, sm_abort(), p, backoff_ns);
     return !barrier_or(kBarIdWorkers, kWorkers, !ok);
 }
 __device__ __forceinline__ bool workers_wait_cluster(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
@@ -512,64 +512,65 @@ struct Worker {
 
     // Softmax of tile i: p = 2^(s c - m) against the running max m, which is raised (with
     // a rescale of O^T and of the sums) only when a score exceeds it by more than
-    // kRescaleThreshold; P^T is written as bf16 hi + lo terms.
+    // kRescaleThreshold; P^T is written as bf16 hi + lo terms.  The scores are read from
+    // tensor memory once; the running sums, which the PV does not read, are updated
+    // after P^T has been handed to the tensor core.
     __device__ __forceinline__ bool softmax(int i) {
-        const int sb = i & 1;
-        if (!workers_wait(&sm_bars()[kBarSFull + sb], (i >> 1) & 1, p, t)) return false;
+        // the tensor core is idle until P^T is written: wake up without backoff
+        if (!workers_wait(&sm_bars()[kBarSFull + (i & 1)], (i >> 1) & 1, p, t, true, 0u)) return false;
         tc_fence_after_sync();
         const float c = p.scale_log2;
         const bool valid = (sm_mask()[(i & 3) * 4 + q] >> lane) & 1u;
         const uint32_t s_col = tmem + lane_base + kTmemS + 16 * hq;
-        const float4 *hm4 = reinterpret_cast<const float4 *>(sm_head_m() + 16 * hq);
+        const float *hm = sm_head_m() + 16 * hq;
+        float x[16], mm[16];
+        tmem_ld16(s_col, x);
+        load16(hm, mm);
+        tmem_wait_ld();
         // does any score exceed its head's running max by more than the threshold?
         bool over = false;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float x[8];
-            tmem_ld8(s_col + 8 * half, x);
-            const float4 m0 = hm4[2 * half], m1 = hm4[2 * half + 1];
-            const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 8; ++h) over |= valid && (x[h] * c - mm[h]) > kRescaleThreshold;
+        for (int h = 0; h < 16; ++h) {
+            x[h] = valid ? x[h] * c : -INFINITY;
+            over |= (x[h] - mm[h]) > kRescaleThreshold;
         }
-        if (barrier_or(kBarIdWorkers, kWorkers, over)) rescale(i, valid, s_col);
-        // p = 2^(s c - m): add to the sums, write P^T row r as bf16 hi + lo, 8 heads at a time
+        if (barrier_or(kBarIdWorkers, kWorkers, over)) {
+            rescale(i, valid, s_col);
+            load16(hm, mm);
+        }
+        // p = 2^(s c - m) (0 for a masked token); P^T row r as bf16 hi + lo
         const int r = 32 * q + lane;
         const uint32_t phi = smem_addr(g_smem + kSmemPhi), plo = smem_addr(g_smem + kSmemPlo);
 #pragma unroll
+        for (int h = 0; h < 16; ++h) x[h] = valid ? fast_exp2(x[h] - mm[h]) : 0.0f;
+#pragma unroll
         for (int half = 0; half < 2; ++half) {
-            const uint32_t l_col = tmem + lane_base + kTmemL + 16 * hq + 8 * half;
-            float x[8], l[8];
-            tmem_ld8(s_col + 8 * half, x);
-            if (i > 0) tmem_ld8(l_col, l);
-            const float4 m0 = hm4[2 * half], m1 = hm4[2 * half + 1];
-            const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-            tmem_wait_ld();
             uint32_t hw[4], lw[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                float a[2];
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int h = 2 * e + k;
-                    a[k] = valid ? fast_exp2(x[h] * c - mm[h]) : 0.0f;
-                    l[h] = (i > 0) ? l[h] + a[k] : a[k];
-                }
+                const float a0 = x[8 * half + 2 * e], a1 = x[8 * half + 2 * e + 1];
                 // hi = the top 16 bits of p (exact bf16), lo = bf16(p - hi): ~16 significant bits
-                hw[e] = pack_bf16x2_trunc(a[0], a[1]);
-                lw[e] = pack_bf16x2(a[0] - __uint_as_float(hw[e] << 16), a[1] - __uint_as_float(hw[e] & 0xFFFF0000u));
+                hw[e] = pack_bf16x2_trunc(a0, a1);
+                lw[e] = pack_bf16x2(a0 - __uint_as_float(hw[e] << 16), a1 - __uint_as_float(hw[e] & 0xFFFF0000u));
             }
-            tmem_st8(l_col, l);
             const uint32_t off = r * 128 + (((2 * hq + half) ^ (r & 7)) << 4);
             sts_v4(phi + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
             sts_v4(plo + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
         }
         fence_proxy_async_smem();
-        tmem_wait_st();
-        tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm_bars()[kBarPFull]);
+        // running sums (per token lane and head) += p
+        const uint32_t l_col = tmem + lane_base + kTmemL + 16 * hq;
+        if (i > 0) {
+            float l[16];
+            tmem_ld16(l_col, l);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h) x[h] += l[h];
+        }
+        tmem_st16(l_col, x);
+        tmem_wait_st();
         return true;
     }
 
