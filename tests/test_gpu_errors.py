@@ -50,16 +50,28 @@ def test_invalid_arguments_rejected_without_launch():
     assert smla.read_error(ws) == 0
 
 
-def test_wait_timeout_reports_and_context_survives():
-    w = W.make_config(2)
+@pytest.mark.parametrize("nsplit", [1, 2, 3, 16])
+def test_wait_timeout_reports_poisons_and_context_survives(nsplit):
+    # The debug hook sends tile 0's S^T commit elsewhere, so every CTA's workers run out of
+    # their 2 ms wait.  Such a call must flag the timeout AND leave its out/lse rows NaN
+    # through every merge path: direct (1 split), the pair's atomic adds (2), the cluster
+    # exchange (3) and the partials + combine kernel (16).  The next call is normal.
+    if nsplit == 16:
+        w = W.make_custom(1, 2048, [100000], seed=11, fill="referenced")
+    else:
+        w = W.make_config(2)
     d = device_inputs(w)
-    ws = smla.binding.new_workspace(w.B, w.topk, nsplit=1)
+    ws = smla.binding.new_workspace(w.B, w.topk, nsplit=nsplit)
     args = (d["q"], d["kv_cache"], d["block_table"], d["topk_idx"], d["seq_lens"], d["sm_scale"])
-    smla.decode(*args, workspace=ws, nsplit=1, wait_timeout_ns=2_000_000,
+    out = torch.zeros((w.B, 64, 512), device="cuda")
+    lse = torch.zeros((w.B, 64), device="cuda")
+    smla.decode(*args, out=out, lse=lse, workspace=ws, nsplit=nsplit, wait_timeout_ns=2_000_000,
                 debug_flags=smla.SMLA_DEBUG_SKIP_FIRST_COMMIT)
+    torch.cuda.synchronize()
     flags = smla.read_error(ws)
     assert flags & smla.SMLA_FLAG_TIMEOUT
-    out, lse = smla.decode(*args, workspace=ws, nsplit=1)
+    assert torch.isnan(out).all() and torch.isnan(lse).all()
+    out, lse = smla.decode(*args, workspace=ws, nsplit=nsplit)
     assert smla.read_error(ws) == 0
     ro, rl = oracle.decode(w.q[0], w.cache, w.block_table, w.topk_idx[0], w.seq_lens, w.sm_scale)
     parity(out, lse, ro, rl)

@@ -43,8 +43,12 @@ def test_config_parity(k):
     print(f"config{k}: nsplit={smla.num_splits(w.B, w.topk)} {figs}")
 
 
-@pytest.mark.parametrize("k", [1, 2, 3])
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 5])
 def test_gather_bit_exact(k):
+    # Index -> (page, slot) translation and dequantisation, bit for bit.  The decode kernel
+    # translates every tile with the same two device helpers as this debug gather
+    # (slot_in_range, then slot_code on the block-table entry), and its UE8M0 dequant is the
+    # same dequant16: configs 4 and 5 cover the large page pools (65 536 and ~8 192 slots).
     w = W.make_config(k)
     d = device_inputs(w)
     lat, ps = smla.debug_gather(d["kv_cache"], d["block_table"], d["topk_idx"], d["seq_lens"])
@@ -78,6 +82,30 @@ def test_gather_scale_extremes_bit_exact():
     assert np.array_equal(np.isnan(g), np.isnan(expect))
     ok = ~np.isnan(expect)
     assert np.array_equal(g[ok], expect[ok])
+
+
+# The validation runs of "The Moment of Validation: A Custom MMA Sparse-Decode Kernel Passes
+# Correctness" (the table of its third attempt): B in {1, 4, 16, 32} x topk in {128, 512}, H = 64,
+# each with len=0 and len=1.  Read here as: len=0 uniform lengths (every request has at least
+# topk tokens, distinct indices, no -1), len=1 ragged lengths (some requests shorter than topk,
+# their tails -1) with scattered -1 slots.  The default split count is used.
+@pytest.mark.parametrize("B", [1, 4, 16, 32])
+@pytest.mark.parametrize("topk", [128, 512])
+@pytest.mark.parametrize("ragged", [0, 1])
+def test_validation_matrix(B, topk, ragged):
+    rng = np.random.default_rng(7000 + 100 * B + topk + ragged)
+    if ragged:
+        seq = rng.integers(1, 3 * topk, size=B)
+        seq[0] = max(1, topk // 3)  # at least one request below topk
+        w = W.make_custom(B, topk, seq, seed=int(rng.integers(1 << 30)), fill="referenced", pad_fraction=0.1)
+    else:
+        seq = rng.integers(topk, 8 * topk, size=B)
+        w = W.make_custom(B, topk, seq, seed=int(rng.integers(1 << 30)), fill="referenced")
+        assert np.all(w.topk_idx[0] >= 0)
+    out, lse, _ = _run(w)
+    ro, rl = _oracle(w)
+    figs = parity(out, lse, ro, rl)
+    print(f"B={B} topk={topk} len={ragged}: nsplit={smla.num_splits(B, topk)} {figs}")
 
 
 @pytest.mark.parametrize("nsplit", [1, 2, 3, 4])

@@ -31,29 +31,62 @@ def _close(o, l, ro, rl):
     assert np.abs(l[fin] - rl[fin]).max() <= LSE_MAX_ABS
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
-    assert torch.cuda.is_available()
+def _noalloc_fn():
     lib = ctypes.CDLL(build.build())
     P, I = ctypes.c_void_p, ctypes.c_int
     fn = lib.smla_decode_noalloc
     fn.argtypes = [P, P, P, P, P, ctypes.c_float, P, P, I, I, I, I, I, P]
     fn.restype = I
-    stream = torch.cuda.current_stream()
-    # two calls in a row: split-K partials (B=64 -> 2 splits, B=1 -> 4 splits) live in the shared scratch
-    for k in (4, 2):
-        w = W.make_config(k)
+    return fn
+
+
+def _call(fn, w, d, out, lse, H=64):
+    return fn(d["q"].data_ptr(), d["kv_cache"].data_ptr(), d["block_table"].data_ptr(), d["topk_idx"].data_ptr(),
+              d["seq_lens"].data_ptr(), ctypes.c_float(w.sm_scale), out.data_ptr(), lse.data_ptr(), w.B, H,
+              w.topk, w.max_blocks, w.num_pages, torch.cuda.current_stream().cuda_stream)
+
+
+def _workloads():
+    # split-K partials in the one scratch array, through every merge path:
+    #   B=64 topk=512 -> 2 splits (pair merge), B=1 topk=512 -> 4 splits (cluster merge),
+    #   B=1 topk=2048 -> 16 splits (global partials + merge kernel),
+    #   B=29 topk=640 -> 5 splits on 145 CTAs: 19.0 MB of partials, near the 19.4 MB worst case
+    yield W.make_config(4)
+    yield W.make_config(2)
+    yield W.make_custom(1, 2048, [100000], seed=21, fill="referenced")
+    yield W.make_custom(29, 640, [4000 + 97 * b for b in range(29)], seed=22, fill="referenced")
+
+
+def test_noalloc_matches_workspace_entry_point_in_sequence():
+    assert torch.cuda.is_available()
+    fn = _noalloc_fn()
+    seen = set()
+    for w in _workloads():
+        seen.add(smla.num_splits(w.B, w.topk))
         d = device_inputs(w)
         ref_o, ref_l = smla.decode(d["q"], d["kv_cache"], d["block_table"], d["topk_idx"], d["seq_lens"],
                                    d["sm_scale"])
         out = torch.full((w.B, 64, 512), float("nan"), device="cuda")
         lse = torch.full((w.B, 64), float("nan"), device="cuda")
-        rc = fn(d["q"].data_ptr(), d["kv_cache"].data_ptr(), d["block_table"].data_ptr(), d["topk_idx"].data_ptr(),
-                d["seq_lens"].data_ptr(), ctypes.c_float(w.sm_scale), out.data_ptr(), lse.data_ptr(), w.B, 64,
-                w.topk, w.max_blocks, w.num_pages, stream.cuda_stream)
-        assert rc == 0
+        assert _call(fn, w, d, out, lse) == 0
         torch.cuda.synchronize()
         _close(out, lse, ref_o, ref_l)
+    assert seen == {2, 4, 16, 5}
     # bad sizes are rejected before any launch
-    assert fn(d["q"].data_ptr(), d["kv_cache"].data_ptr(), d["block_table"].data_ptr(), d["topk_idx"].data_ptr(),
-              d["seq_lens"].data_ptr(), ctypes.c_float(w.sm_scale), out.data_ptr(), lse.data_ptr(), w.B, 32,
-              w.topk, w.max_blocks, w.num_pages, stream.cuda_stream) == -1
+    assert _call(fn, w, d, out, lse, H=32) == -1
+
+
+def test_noalloc_allocates_nothing():
+    fn = _noalloc_fn()
+    w = W.make_custom(29, 640, [4000 + 97 * b for b in range(29)], seed=22, fill="referenced")
+    d = device_inputs(w)
+    out = torch.empty((w.B, 64, 512), device="cuda")
+    lse = torch.empty((w.B, 64), device="cuda")
+    assert _call(fn, w, d, out, lse) == 0  # warm-up: module load, attributes
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _call(fn, w, d, out, lse) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
