@@ -8,6 +8,12 @@ B=64, topk=512 workload (64 requests of 65536 tokens, 256 pages each, one
 touched, more than 4x the 126 MB L2) so consecutive steps never find their KV
 rows in L2.
 
+The line also carries `per_config`: microseconds per call, algorithmic GB/s and the
+roofline fraction of all five workloads of the sparse MLA decode target (B=1 topk=64;
+B=1 topk=512; B=16 ragged; B=64; B=256), each timed on its own: B=64 and B=256 as
+CUDA graphs over rotating replicas (more than 4x L2 per rotation), the three small
+ones per call between L2 flushes (their whole page pools are at most 121 MB).
+
 Modes:
   python bench.py [--gpus N] [--steps K] [--warmup W]      # CUDA path
   python bench.py --impl reference ...                     # the fp64 oracle on the host cores
@@ -170,6 +176,109 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+CONFIG_LABELS = {1: "B=1 topk=64 (launch-bound: a few us of work)", 2: "B=1 topk=512 (launch-bound: 4 CTAs)",
+                 3: "B=16 topk=512, ragged seq_len in [256, 32768]", 4: "B=64 topk=512, seq_len 65536, 1% outliers",
+                 5: "B=256 topk=512, seq_len in [1024, 8192], ~2M-token pool"}
+
+
+def _config_entry(k, w, us, nsplit, timing, peaks):
+    from sparse_mla_decode_fp8_b200 import workloads as W
+
+    units = W.roofline_units(w.replica(0))
+    t_hbm = units["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_tc = units["flops"] / (peaks["bf16_tflops"] * 1e12) * 1e6
+    gbs = units["bytes"] / (us * 1e-6) / 1e9
+    return {"workload": CONFIG_LABELS[k], "B": w.B, "topk": w.topk, "nsplit": nsplit, "us_per_call": us,
+            "algorithmic_bytes": units["bytes"], "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+            "roofline_us": max(t_hbm, t_tc), "frac_of_roofline": max(t_hbm, t_tc) / us,
+            "tc_tflops": units["flops"] / (us * 1e-6) / 1e12, "timing": timing}
+
+
+def time_small_config(k, dev, peaks, calls: int = 40):
+    """Per-call CUDA-event time of one small workload, 512 MB written between calls to flush L2."""
+    import torch
+
+    import sparse_mla_decode_fp8_b200 as smla
+    from sparse_mla_decode_fp8_b200 import workloads as W
+
+    w = W.make_config(k)
+    q = torch.from_numpy(np.ascontiguousarray(w.q[0]).view(np.int16)).view(torch.bfloat16).to(dev)
+    cache = torch.from_numpy(w.cache).to(dev)
+    bt = torch.from_numpy(w.block_table).to(dev)
+    idx = torch.from_numpy(np.ascontiguousarray(w.topk_idx[0])).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    nsplit = smla.num_splits(w.B, w.topk)
+    ws = torch.zeros(smla.workspace_bytes(w.B, w.topk), dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, 64, 512), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, 64), dtype=torch.float32, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            smla.decode(q, cache, bt, idx, sl, w.sm_scale, out=out, lse=lse, workspace=ws, stream=stream)
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(stream)
+            smla.decode(q, cache, bt, idx, sl, w.sm_scale, out=out, lse=lse, workspace=ws, stream=stream)
+            b.record(stream)
+    stream.synchronize()
+    assert smla.read_error(ws, stream) == 0
+    us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+    timing = f"median of {calls} calls, CUDA events around each, 512 MB written between calls (L2 flush)"
+    return _config_entry(k, w, us, nsplit, timing, peaks)
+
+
+def time_rotating_config(k, w, dev, peaks, calls: int = 200, reps: int = 5):
+    """CUDA-graph time per call of a large workload over its rotating replicas."""
+    import torch
+
+    import sparse_mla_decode_fp8_b200 as smla
+
+    cache = torch.from_numpy(w.cache).to(dev)
+    bt = torch.from_numpy(w.block_table).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    qs = [torch.from_numpy(np.ascontiguousarray(w.q[r]).view(np.int16)).view(torch.bfloat16).to(dev)
+          for r in range(w.R)]
+    idxs = [torch.from_numpy(np.ascontiguousarray(w.topk_idx[r])).to(dev) for r in range(w.R)]
+    nsplit = smla.num_splits(w.B, w.topk)
+    ws = torch.zeros(smla.workspace_bytes(w.B, w.topk), dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, 64, 512), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, 64), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        r = i % w.R
+        smla.decode(qs[r], cache, bt, idxs[r], sl, w.sm_scale, out=out, lse=lse, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(calls):
+            step(i)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    assert smla.read_error(ws, stream) == 0
+    us = e0.elapsed_time(e1) * 1e3 / (calls * reps)
+    from sparse_mla_decode_fp8_b200 import workloads as W
+
+    per_rot = W.roofline_units(w.replica(0))["bytes"] * w.R
+    timing = (f"CUDA graph of {calls} calls over {w.R} rotating replicas ({per_rot / 1e6:.0f} MB of KV+Q per "
+              f"rotation > 4x L2), replayed {reps}x, CUDA events")
+    del g
+    return _config_entry(k, w, us, nsplit, timing, peaks)
 
 
 def max_over_ranks(value: float, dist=None, device=None) -> float:
@@ -358,6 +467,15 @@ def run_cuda(args):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
+    if not args.no_per_config:
+        per = {}
+        for k in (1, 2, 3):
+            per[f"config{k}"] = time_small_config(k, dev, peaks)
+        per["config4"] = _config_entry(4, w, call_ms * 1e3, nsplit, line["config"]["timing"] + " (the headline run)",
+                                       peaks)
+        w5 = W.make_config(5, replicas=8)
+        per["config5"] = time_rotating_config(5, w5, dev, peaks)
+        line["per_config"] = per
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_baseline(w, min_seconds=args.cpu_seconds, max_reps=200)
     print(json.dumps(line), flush=True)
@@ -399,6 +517,7 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="time only the headline workload")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -55,9 +55,11 @@ constexpr int kCtlWarp = kWorkerWarps;         // warp 16: tensor memory, mbarri
 constexpr int kThreads = kWorkers + 32;        // 544 threads: at most 120 registers each
 constexpr int kGatherThreads = 256;            // threads of the gather debug kernel
 constexpr uint32_t kBarIdWorkers = 1;          // named barrier of the 512 worker threads
-constexpr uint32_t kBarIdHeads = 2;            // named barrier of worker threads 0..63 (one per head)
 constexpr int kWaiter = 32;                    // the worker that waits on behalf of all workers
-constexpr int kMaxClusterSplits = 4;           // splits of a request that merge inside a cluster
+// Two splits of a request merge inside the kernel (a CTA pair in one cluster, two terms
+// per output element: the sum does not depend on their order); more go through global
+// partials and the merge kernel, whose fixed order keeps the result reproducible.
+constexpr int kMaxClusterSplits = 2;
 
 // Dynamic shared memory map (bytes from a 1024-aligned base).
 constexpr int kSmemQ = 0;                         // 64 KB: 8 K-blocks x [64 heads x 128 B], TMA-written
@@ -80,11 +82,8 @@ enum Bar : int {
     kBarPFull = 11,     // P^T written (16 worker-warp arrivals)
     kBarDrain = 12,     // final commit before tensor memory is released
     kBarSpare = 13,     // test hook target
-    kBarMl = 14,        // cluster merge: the peers' (m, l) rows are in (3-4 splits: the workspace, one arrival
-                        // per peer; 2 splits: the peer's log-sum-exp row, 256 transaction bytes)
-    kBarRxReady = 15,   // cluster merge: every peer's receive buffer is free (one arrival per peer)
-    kBarRx = 16,        // + k (k = 0..3): owned output unit k received (one arrival per sending lane)
-    kNumBars = 20,
+    kBarMl = 14,        // pair merge: the peer's log-sum-exp row is in (256 transaction bytes)
+    kNumBars = 15,
 };
 constexpr int kSmemTmemSlot = kSmemBars + kNumBars * 8;
 constexpr int kSmemAbort = kSmemTmemSlot + 4;
@@ -113,13 +112,6 @@ constexpr uint32_t kIdescPV2 = idesc_bf16(128, 128, true, true);
 // pass over O^T in tensor memory) rare after the first tile, even when a few latents are
 // much larger than the rest.
 constexpr float kRescaleThreshold = 64.0f;
-
-// Split merge inside a cluster: the 512 output dims form 8 units of 64; unit u belongs
-// to CTA u % nsplit.  A CTA receives its units' partials from every peer into 16 KB
-// slots ([64 dims][64 heads] f32, 16-byte groups of 4 heads swizzled by dim & 7):
-// in the Q buffer (free after the last score MMA) when nsplit = 2, else in the KV
-// buffer (free after the last PV).
-constexpr int kUnitBytes = 64 * kHeads * 4;
 
 // The CTA's dynamic shared memory.  Every function addresses it through these
 // accessors (constant offsets from the shared window), so no 64-bit pointer to
@@ -229,20 +221,6 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
     return ok != 0;
 }
 
-// Bounded wait on a phase completed by other CTAs of the cluster (acquire at cluster
-// scope); every calling thread observes the phase itself.
-__device__ __noinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parity, const DecodeParams &p) {
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t k = 1;; ++k) {
-        if (mbar_test_wait_cluster(bar, parity)) return true;
-        __nanosleep(kWorkerBackoffNs);
-        if ((k & 31u) == 0 && global_timer_ns() - t0 > p.timeout_ns) {
-            atomicOr(p.err, SMLA_FLAG_TIMEOUT);
-            return false;
-        }
-    }
-}
-
 // Worker-wide waits: one worker thread (in warp 1, so it does not share a scheduler
 // with the MMA-issuing warp 16) waits on the mbarrier phase, with acquire semantics,
 // while the other workers block in a named barrier; the barrier then orders every
@@ -254,12 +232,6 @@ __device__ __forceinline__ bool workers_wait(uint64_t *bar, uint32_t parity, con
                                              bool enabled = true, uint32_t backoff_ns = kWorkerBackoffNs) {
     bool ok = enabled;
     if (t == kWaiter && enabled) ok = wait_phase(bar, parity, sm_abort(), p, backoff_ns);
-    return !barrier_or(kBarIdWorkers, kWorkers, !ok);
-}
-__device__ __forceinline__ bool workers_wait_cluster(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
-                                                     bool enabled = true) {
-    bool ok = enabled;
-    if (t == kWaiter && enabled) ok = wait_cluster_phase(bar, parity, p);
     return !barrier_or(kBarIdWorkers, kWorkers, !ok);
 }
 
@@ -794,139 +766,6 @@ __device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) 
     }
 }
 
-// nsplit = 3..4 in one cluster.  With L = log2 sum_s 2^(m_s) l_s over the splits s, the
-// merged output is O = sum_s 2^(m_s - L) O^T_s and LSE = L ln 2 (the split-K
-// log-sum-exp merge).  Every CTA publishes its (m, l) row to the workspace and signals
-// its peers; output unit u (dims [64u, 64u+64)) belongs to CTA u % nsplit.  Chunk by
-// chunk, as the last PV finishes dims chunk c, the warps whose lanes cover a unit of
-// chunk c (u = 2c + q/2) that another CTA owns store their O^T values into the owner's
-// receive slot (distributed shared memory) and signal it with one arrival per lane;
-// the owner warps wait for every peer's values of their unit and write the merged
-// output.
-__device__ __forceinline__ void epilogue_cluster(Worker &w, int b, int n, bool ok) {
-    const DecodeParams &p = w.p;
-    const int ns = p.nsplit;
-    const int me = static_cast<int>(cluster_ctarank());
-    const int t = w.t;
-    uint64_t *bars = sm_bars();
-    float *ml = p.part_lse + static_cast<size_t>(b) * ns * 128;
-    const int rx_base = (ns == 2) ? kSmemQ : kSmemKV;
-    // 1. publish (m, l) (one arrival per peer once all 64 heads are stored); signal that
-    //    this CTA's receive buffer is free: with nsplit = 2 it is the Q buffer, idle since
-    //    the last score MMA (the softmax of the last tile waited for it), otherwise the KV
-    //    buffer once the last PV is done
-    if (t < kHeads) {
-        __stcg(ml + me * 128 + t, ok ? sm_head_m()[t] : NAN);
-        __stcg(ml + me * 128 + 64 + t, ok ? sm_head_alpha()[t] : NAN);
-        fence_acq_rel_cluster();
-        named_barrier_sync(kBarIdHeads, kHeads);
-        if (t == 0) {
-            for (int s = 0; s < ns; ++s)
-                if (s != me) mbar_arrive_remote(map_to_rank(&bars[kBarMl], s));
-            if (ns > 2 && ok && n > 0) (void)wait_phase(&bars[kBarKvFree + 3], (n - 1) & 1, sm_abort(), p);
-            for (int s = 0; s < ns; ++s)
-                if (s != me) mbar_arrive_remote(map_to_rank(&bars[kBarRxReady], s));
-        }
-    }
-    // 2. merge weights per (split, head)
-    float *weights = sm_red();  // [ns][64]
-    if (t < kHeads) {
-        int got = 1;
-        if (t == 0) got = wait_cluster_phase(&bars[kBarMl], 0, p) ? 1 : 0;
-        got = barrier_or(kBarIdHeads, kHeads, !got) ? 0 : 1;
-        if (got) (void)mbar_try_wait_cluster(&bars[kBarMl], 0);
-        float mv[kMaxClusterSplits], lv[kMaxClusterSplits];
-        bool bad = !got;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < kMaxClusterSplits; ++s) {
-            mv[s] = -INFINITY;
-            lv[s] = 0.0f;
-            if (s < ns) {
-                mv[s] = (s == me) ? (ok ? sm_head_m()[t] : NAN) : __ldcg(ml + s * 128 + t);
-                lv[s] = (s == me) ? (ok ? sm_head_alpha()[t] : NAN) : __ldcg(ml + s * 128 + 64 + t);
-            }
-            bad = bad || isnan(mv[s]) || isnan(lv[s]);
-            if (lv[s] > 0.0f) mx = fmaxf(mx, mv[s]);
-        }
-        float sum = 0.0f;
-#pragma unroll
-        for (int s = 0; s < kMaxClusterSplits; ++s)
-            if (lv[s] > 0.0f) sum += exp2f(mv[s] - mx) * lv[s];
-        const float L = (sum > 0.0f) ? mx + log2f(sum) : -INFINITY;
-#pragma unroll
-        for (int s = 0; s < kMaxClusterSplits; ++s)
-            if (s < ns) weights[s * kHeads + t] = bad ? NAN : (sum > 0.0f && lv[s] > 0.0f) ? exp2f(mv[s] - L) : 0.0f;
-        if (me == 0) p.lse[static_cast<size_t>(b) * kHeads + t] = bad ? NAN : (sum > 0.0f) ? L * 0.69314718055994531f
-                                                                                               : -INFINITY;
-    }
-    // the peers' receive buffers must be free before anything is sent (this barrier also
-    // publishes the weights)
-    const bool rx_ready = workers_wait_cluster(&bars[kBarRxReady], 0, p, t);
-    // 3. stream the units chunk by chunk as the last PV finishes them.  Each warp runs
-    //    its own loop: the unit of chunk c it covers depends only on c and on the peer
-    //    warps with the same index, which send chunk c before they wait for anything
-    //    of chunk c+1, so no warp waits on a warp that waits on it.
-    const int d = 32 * (w.q & 1) + w.lane;  // dim within the unit
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        const int u = 2 * c + (w.q >> 1);
-        const int o = u % ns;
-        const bool chunk_ok =
-            ok && n > 0 && warp_wait_phase(&bars[kBarKvFree + c], (n - 1) & 1, sm_abort(), p, w.lane);
-        float v[16];
-        if (chunk_ok) {
-            load_o16(w.tmem + w.lane_base, c, w.hq, v);
-        } else {
-            // no tile (O = 0, weight 0) or a failed wait (the result is invalid)
-#pragma unroll
-            for (int h = 0; h < 16; ++h) v[h] = (ok && n == 0) ? 0.0f : NAN;
-        }
-        if (o != me) {
-            // without rx_ready nothing is sent: the owner's wait runs out and it writes NaN
-            if (rx_ready) {
-                const int slot = (u / ns) * (ns - 1) + (me < o ? me : me - 1);
-                const uint32_t row = map_to_rank(g_smem + rx_base + slot * kUnitBytes + d * 256, o);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int g = (4 * w.hq + j) ^ (d & 7);
-                    st_cluster_v4(row + g * 16, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                }
-                // one arrival per lane, releasing that lane's stores
-                mbar_arrive_remote(map_to_rank(&bars[kBarRx + u / ns], o));
-            }
-            continue;
-        }
-        int got = 1;
-        if (w.lane == 0) got = wait_cluster_phase(&bars[kBarRx + u / ns], 0, p) ? 1 : 0;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (got) (void)mbar_try_wait_cluster(&bars[kBarRx + u / ns], 0);
-        float acc[16], wt[16];
-        load16(weights + me * kHeads + 16 * w.hq, wt);
-#pragma unroll
-        for (int h = 0; h < 16; ++h) acc[h] = (wt[h] != 0.0f) ? v[h] * wt[h] : 0.0f;  // NaN weights propagate
-        for (int s = 0; s < ns; ++s) {
-            if (s == me) continue;
-            const int slot = (u / ns) * (ns - 1) + (s < me ? s : s - 1);
-            const float *row = reinterpret_cast<const float *>(g_smem + rx_base + slot * kUnitBytes + d * 256);
-            load16(weights + s * kHeads + 16 * w.hq, wt);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float4 r = reinterpret_cast<const float4 *>(row)[(4 * w.hq + j) ^ (d & 7)];
-                const float rv[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float ws = wt[4 * j + e];
-                    if (ws != 0.0f) acc[4 * j + e] += rv[e] * ws;
-                }
-            }
-        }
-        float *dst = p.out + (static_cast<size_t>(b) * kHeads + 16 * w.hq) * kDim + 64 * u + d;
-#pragma unroll
-        for (int h = 0; h < 16; ++h) dst[h * kDim] = got ? acc[h] : NAN;
-    }
-}
-
 // ------------------------------------------------------------------ the decode kernel
 // One CTA per (topk split, request).  The 16 worker warps move one 128-slot tile at a
 // time through dequantisation and softmax while the rows of the next two tiles are in
@@ -959,7 +798,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int seq_len = __ldg(p.seq_lens + b);
     const int32_t *bt_row = p.block_table + static_cast<size_t>(b) * p.max_blocks;
     const int32_t *idx_row = p.topk_idx + static_cast<size_t>(b) * p.topk;
-    const int ns = p.nsplit;
 
     // ---- setup
     Translator tr;
@@ -971,17 +809,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) {
                 mbar_init(&bars[kBarKvFull + c], kWorkerWarps);
                 mbar_init(&bars[kBarKvFree + c], 1);
-                mbar_init(&bars[kBarRx + c], p.cluster_merge ? (ns - 1) * 8 * 32 : 1);  // 8 warps per peer
             }
             mbar_init(&bars[kBarSFull], 1);
             mbar_init(&bars[kBarSFull + 1], 1);
             mbar_init(&bars[kBarPFull], kWorkerWarps);
             mbar_init(&bars[kBarDrain], 1);
             mbar_init(&bars[kBarSpare], 1);
-            mbar_init(&bars[kBarMl], (p.cluster_merge && ns > 2) ? ns - 1 : 1);
-            mbar_init(&bars[kBarRxReady], p.cluster_merge ? ns - 1 : 1);
-            // two splits: the peer's row of 64 log-sum-exps arrives as 256 transaction bytes
-            if (p.cluster_merge && ns == 2) mbar_arrive_expect_tx(&bars[kBarMl], kHeads * 4);
+            mbar_init(&bars[kBarMl], 1);
+            // the peer's row of 64 log-sum-exps arrives as 256 transaction bytes
+            if (p.cluster_merge) mbar_arrive_expect_tx(&bars[kBarMl], kHeads * 4);
             fence_barrier_init();
             *sm_abort() = 0;
             mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
@@ -1004,7 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (tid < kHeads) head_m[tid] = -INFINITY;
-    if (p.cluster_merge && ns == 2) {
+    if (p.cluster_merge) {
         // two splits add their weighted partials into the output: each CTA zeroes 32 heads of
         // out[b] now; the barriers below order these stores before either CTA's additions
         float4 *z = reinterpret_cast<float4 *>(p.out + (static_cast<size_t>(b) * kHeads + 32 * split) * kDim);
@@ -1034,11 +870,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = !barrier_or(kBarIdWorkers, kWorkers, !ok);
         w.reduce_sums(ok && n > 0);
         if (p.cluster_merge) {
-            cluster_wait();  // every peer has initialised its mbarriers (and zeroed its part of out)
-            if (ns == 2)
-                epilogue_pair(w, b, n, ok);
-            else
-                epilogue_cluster(w, b, n, ok);
+            cluster_wait();  // the peer has initialised its mbarriers and zeroed its half of out
+            epilogue_pair(w, b, n, ok);
         } else {
             epilogue_direct(w, b, split, n, ok);
         }
@@ -1245,20 +1078,17 @@ bool sizes_ok(int B, int H, int topk) {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Up to smla::kMaxClusterSplits splits of a request merge inside a thread-block cluster
-// (partial outputs travel through distributed shared memory); beyond it they go
-// through normalised global partials and the merge kernel.
+// Two splits of a request merge inside the decode kernel (a CTA pair: the log-sum-exp
+// rows cross through distributed shared memory, the outputs are added into out); more
+// go through normalised global partials and the merge kernel.
 //
-// Workspace after the header: nsplit == 1: nothing.  2..4 (cluster merge): the
-// per-split (m, l) rows [B][nsplit][128] f32.  Above 4: part_lse [B][64][nsplit]
+// Workspace after the header: nsplit <= 2: nothing.  Above 2: part_lse [B][64][nsplit]
 // f32, then part_o [B][64][nsplit][512] f32.
 size_t workspace_for(int B, int topk, int nsplit) {
     size_t bytes = SMLA_WORKSPACE_HEADER;
     if (nsplit > smla::kMaxClusterSplits) {
         const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
         bytes += round256(rows * sizeof(float)) + rows * SMLA_DIM * sizeof(float);
-    } else if (nsplit > 1) {
-        bytes += round256(static_cast<size_t>(B) * nsplit * 128 * sizeof(float));
     }
     (void)topk;
     return bytes;
@@ -1333,10 +1163,11 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     p.lse = lse;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.err = reinterpret_cast<uint32_t *>(ws);
-    const size_t rows = (nsplit > smla::kMaxClusterSplits) ? static_cast<size_t>(B) * SMLA_HEADS * nsplit
-                                                           : static_cast<size_t>(B) * nsplit * 128;
-    p.part_lse = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER);
-    p.part_o = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER + round256(rows * sizeof(float)));
+    if (nsplit > smla::kMaxClusterSplits) {
+        const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
+        p.part_lse = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER);
+        p.part_o = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER + round256(rows * sizeof(float)));
+    }
     p.num_pages = num_pages;
     p.timeout_ns = (opts && opts->wait_timeout_ns) ? opts->wait_timeout_ns : 1000000000ull;
     p.topk = topk;
