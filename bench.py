@@ -53,9 +53,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_desc(w):
-    return (f"config{CONFIG}: B={w.B} H={w.H} topk={w.topk} seq_len=65536 (256 pages/request, "
-            f"{w.num_pages}-page pool), e4m3 nope + UE8M0 per 64 + bf16 rope, 1% outlier rows x20, "
+def workload_desc(w, k=CONFIG):
+    if k == 4:
+        return (f"config4: B={w.B} H={w.H} topk={w.topk} seq_len=65536 (256 pages/request, "
+                f"{w.num_pages}-page pool), e4m3 nope + UE8M0 per 64 + bf16 rope, 1% outlier rows x20, "
+                f"sm_scale=512^-0.5")
+    return (f"config{k}: {CONFIG_LABELS[k]}, {w.num_pages}-page pool, e4m3 nope + UE8M0 per 64 + bf16 rope, "
             f"sm_scale=512^-0.5")
 
 
@@ -141,7 +144,7 @@ def run_reference(args):
     from sparse_mla_decode_fp8_b200 import workloads as W
 
     oracle.build()
-    w = W.make_config(CONFIG, replicas=1)
+    w = W.make_config(args.config, replicas=1)
     all_rows = np.array([(b, h) for b in range(w.B) for h in range(w.H)], np.int32)
     # calibrate: seconds per (b, h) row when a step holds one request's 64 rows
     t0 = time.perf_counter()
@@ -169,7 +172,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": max(1, args.steps), "warmup": args.warmup, "ms_per_step": 1e3 * el / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(w), "B": w.B, "topk": w.topk, "H": w.H,
+            "config": {"workload": workload_desc(w, args.config), "B": w.B, "topk": w.topk, "H": w.H,
                        "parallelism": "host cores (OpenMP over requests)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
@@ -321,7 +324,7 @@ def run_cuda(args):
     smla_build.build()
     smla.library()
 
-    w = W.make_config(CONFIG, replicas=REPLICAS, seed=None if rank == 0 else 1000 + rank)
+    w = W.make_config(args.config, replicas=REPLICAS, seed=None if rank == 0 else 1000 + rank)
     B, topk, H = w.B, w.topk, w.H
     cache = torch.from_numpy(w.cache).to(dev)
     bt = torch.from_numpy(w.block_table).to(dev)
@@ -441,13 +444,13 @@ def run_cuda(args):
     achieved_tf = units["flops"] / (call_ms * 1e-3) / 1e12
     t_hbm_us = units["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_tc_us = units["flops"] / (peaks["bf16_tflops"] * 1e12) * 1e6
-    traffic = _profiled_traffic()
+    traffic = _profiled_traffic(args.config)
     line = {
         "metric": METRIC, "value": job_throughput(world, B, topk, steps, max_ms), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step, "us_per_call": ms_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload_desc(w), "B": B, "topk": topk, "H": H, "nsplit": nsplit,
+        "config": {"workload": workload_desc(w, args.config), "B": B, "topk": topk, "H": H, "nsplit": nsplit,
                    "l2": f"inputs larger than L2: {REPLICAS} rotating replicas, "
                          f"{REPLICAS * units['bytes'] / 1e6:.0f} MB of KV+Q touched per rotation > 126 MB",
                    "parallelism": f"replicas x{world} (no collective)", "timing": f"CUDA graph of {gsteps} steps "
@@ -467,7 +470,7 @@ def run_cuda(args):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
-    if not args.no_per_config:
+    if not args.no_per_config and args.config == CONFIG:
         per = {}
         for k in (1, 2, 3):
             per[f"config{k}"] = time_small_config(k, dev, peaks)
@@ -482,9 +485,14 @@ def run_cuda(args):
     return 0
 
 
-def _profiled_traffic():
+PROFILES = {4: "decode_kernel_B64_topk512.md", 5: "decode_kernel_B256_topk512.md"}
+
+
+def _profiled_traffic(k: int):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_kernel_config4.md")
+    if k not in PROFILES:
+        return None
+    path = os.path.join(ROOT, "profiles", PROFILES[k])
     if not os.path.exists(path):
         return None
     fields = {}
@@ -518,6 +526,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="time only the headline workload")
+    ap.add_argument("--config", type=int, default=CONFIG, choices=[3, 4, 5],
+                    help="workload of the timed run (default: the B=64 headline); 3 and 5 for profiling")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
