@@ -59,6 +59,16 @@ def _bind(path: str):
     lib.orc_decode.restype = ctypes.c_int
     lib.orc_combine.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
     lib.orc_combine.restype = ctypes.c_int
+    lib.orc_e4m3_encode.argtypes = [ctypes.c_double]
+    lib.orc_e4m3_encode.restype = ctypes.c_uint8
+    lib.orc_bf16_encode.argtypes = [ctypes.c_float]
+    lib.orc_bf16_encode.restype = ctypes.c_uint16
+    lib.orc_scale_exponent.argtypes = [P]
+    lib.orc_scale_exponent.restype = ctypes.c_int
+    lib.orc_quantize_token.argtypes = [P, P, P]
+    lib.orc_quantize_token.restype = None
+    lib.orc_write_kv.argtypes = [P, ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int64, P]
+    lib.orc_write_kv.restype = ctypes.c_int
     return lib
 
 
@@ -176,3 +186,47 @@ def combine(part_o, part_lse, lib=None):
     if rc != 0:
         raise ValueError("orc_combine rejected its arguments")
     return out, lse
+
+
+def e4m3_encode(x: float, lib=None) -> int:
+    """e4m3 (fn) code nearest to x (ties to the even code); |x| >= 448 saturates; NaN -> 0x7F."""
+    return int((lib or _load()).orc_e4m3_encode(float(x)))
+
+
+def bf16_encode(x: float, lib=None) -> int:
+    """bf16 bits of a binary32 value, round to nearest even; NaN -> 0x7FC0."""
+    return int((lib or _load()).orc_bf16_encode(float(np.float32(x))))
+
+
+def scale_exponent(group, lib=None) -> int:
+    """Scale exponent e of one 64-value nope group: the smallest e with max|x| <= 448 * 2^e,
+    clamped to [-127, 127] (-127 when all zero, 127 when a value is not finite)."""
+    g = _c(group, np.float32)
+    assert g.shape == (64,)
+    return int((lib or _load()).orc_scale_exponent(_ptr(g)))
+
+
+def quantize_token(latent, lib=None):
+    """One 512-d fp32 latent -> (576-byte row, 8-byte scale row): the cache format of "The
+    Validation Gate" ("The Test Design"), per 64-dim UE8M0 scale and e4m3 nope, bf16 rope."""
+    x = _c(latent, np.float32)
+    assert x.shape == (DIM,)
+    row = np.zeros(576, np.uint8)
+    sc = np.zeros(8, np.uint8)
+    (lib or _load()).orc_quantize_token(_ptr(x), _ptr(row), _ptr(sc))
+    return row, sc
+
+
+def write_kv(latents, req, pos, block_table, cache, lib=None) -> int:
+    """Quantise latents [n,512] and store each at position pos[i] of request req[i]
+    (page = block_table[req][pos // 256], slot = pos % 256), in place in ``cache``
+    [pages, PAGE_BYTES] uint8.  Out-of-range destinations are skipped; returns their count."""
+    x = _c(latents, np.float32).reshape(-1, DIM)
+    r = _c(req, np.int32)
+    p = _c(pos, np.int32)
+    bt = _c(block_table, np.int32)
+    assert cache.dtype == np.uint8 and cache.flags["C_CONTIGUOUS"] and cache.shape[-1] == PAGE_BYTES
+    n = x.shape[0]
+    assert r.shape == (n,) and p.shape == (n,)
+    return int((lib or _load()).orc_write_kv(_ptr(x), n, _ptr(r), _ptr(p), _ptr(bt), bt.shape[0], bt.shape[1],
+                                             cache.shape[0], _ptr(cache)))

@@ -264,3 +264,107 @@ int orc_combine(const double *part_o, const double *part_lse, int B, int H, int 
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ cache writer
+ * The inverse of orc_token_latent, for the synthetic-cache quantisation the pages
+ * leave open (reading: scale exponent e = ceil(log2(amax / 448)) per 64-dim nope
+ * group, i.e. the smallest e with amax <= 448 * 2^e, clamped to [-127, 127] and -127
+ * for an all-zero group; scale byte e + 127; nope byte = e4m3 of x / 2^e rounded to
+ * nearest, ties to even; rope = bf16 of x rounded to nearest, ties to even).
+ * Non-finite inputs (not produced by the generators; fixed here so that two writers
+ * can be compared byte for byte): a group holding an infinity or NaN takes e = 127;
+ * +-inf saturates to +-448, NaN becomes 0x7F; a NaN rope value becomes 0x7FC0. */
+
+/* Nearest e4m3 (fn) code to x by search over the 127 non-negative finite codes; a
+ * tie goes to the code whose last mantissa bit is 0; |x| >= 448 gives 448 (0x7E). */
+uint8_t orc_e4m3_encode(double x) {
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x), best_d = INFINITY;
+    int c, best = 0;
+    if (isnan(x)) return 0x7F;
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    for (c = 0; c <= 0x7E; c++) {
+        double d = fabs(orc_e4m3((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best_d = d;
+            best = c;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* bf16 of a binary32 value: the nearer of the two bf16 values around it (its upper
+ * half truncated, and the next one away from zero), a tie to the one whose last bit
+ * is 0.  The truncation is exact for values that are already bf16. */
+uint16_t orc_bf16_encode(float f) {
+    uint32_t bits;
+    uint16_t lo, hi;
+    double dlo, dhi, v = (double)f;
+    if (isnan(f)) return 0x7FC0;
+    memcpy(&bits, &f, sizeof bits);
+    lo = (uint16_t)(bits >> 16);
+    if ((bits & 0xFFFF) == 0) return lo;
+    hi = (uint16_t)(lo + 1); /* next magnitude up; past the largest finite it is the infinity, */
+    dlo = fabs(orc_bf16(lo) - v); /* which rounding treats as the value 2^128 */
+    dhi = ((hi & 0x7FFF) == 0x7F80) ? fabs(copysign(ldexp(1.0, 128), v) - v) : fabs(orc_bf16(hi) - v);
+    if (dlo < dhi) return lo;
+    if (dhi < dlo) return hi;
+    return (lo & 1) ? hi : lo;
+}
+
+/* The scale exponent of one nope group (see the reading above). */
+int orc_scale_exponent(const float *x) {
+    double amax = 0.0;
+    int d, e;
+    for (d = 0; d < ORC_GROUP; d++) {
+        if (!isfinite(x[d])) return 127;
+        if (fabs((double)x[d]) > amax) amax = fabs((double)x[d]);
+    }
+    if (amax == 0.0) return -127;
+    e = -127;
+    while (e < 127 && ldexp(448.0, e) < amax) e++;
+    return e;
+}
+
+/* One 512-d latent -> its 576-byte row and 8-byte scale row (byte 7 = 0). */
+void orc_quantize_token(const float *x, uint8_t *row, uint8_t *scale_row) {
+    int g, d, r;
+    for (g = 0; g < ORC_NOPE / ORC_GROUP; g++) {
+        int e = orc_scale_exponent(x + g * ORC_GROUP);
+        scale_row[g] = (uint8_t)(e + 127);
+        for (d = g * ORC_GROUP; d < (g + 1) * ORC_GROUP; d++) row[d] = orc_e4m3_encode(ldexp((double)x[d], -e));
+    }
+    scale_row[ORC_NOPE / ORC_GROUP] = 0;
+    for (r = 0; r < ORC_ROPE; r++) {
+        uint16_t u = orc_bf16_encode(x[ORC_NOPE + r]);
+        row[ORC_NOPE + 2 * r] = (uint8_t)(u & 0xFF);
+        row[ORC_NOPE + 2 * r + 1] = (uint8_t)(u >> 8);
+    }
+}
+
+/* Writes n latents [n,512] at positions pos[i] of requests req[i]: page =
+ * block_table[req][pos / 256], slot = pos % 256 (the page indexing of "The
+ * Validation Moment").  A token whose request, position or page is out of range
+ * is skipped.  Returns the number of skipped tokens. */
+int orc_write_kv(const float *latents, int n, const int32_t *req, const int32_t *pos,
+                 const int32_t *block_table, int B, int max_blocks, int64_t num_pages, uint8_t *cache) {
+    int i, skipped = 0;
+    for (i = 0; i < n; i++) {
+        int32_t b = req[i], p = pos[i], page;
+        uint8_t *page_base;
+        if (b < 0 || b >= B || p < 0 || p / ORC_PAGE_TOKENS >= max_blocks) {
+            skipped++;
+            continue;
+        }
+        page = block_table[(int64_t)b * max_blocks + p / ORC_PAGE_TOKENS];
+        if (page < 0 || (int64_t)page >= num_pages) {
+            skipped++;
+            continue;
+        }
+        page_base = cache + (int64_t)page * ORC_PAGE_BYTES;
+        orc_quantize_token(latents + (int64_t)i * ORC_DIM,
+                           page_base + (int64_t)(p % ORC_PAGE_TOKENS) * ORC_ROW_BYTES,
+                           page_base + ORC_SCALE_BLOCK_OFFSET + (int64_t)(p % ORC_PAGE_TOKENS) * ORC_SCALE_ROW_BYTES);
+    }
+    return skipped;
+}

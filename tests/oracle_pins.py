@@ -15,6 +15,11 @@ What pins what:
     gives the mean; all slots equal), invariances (permutation, -1 slots,
     multiplicity), a dense masked brute force decoded through torch dtypes, and
     the LSE-merge identity for the combine.
+  * cache writer -- the e4m3 / bf16 encoders against torch's float8_e4m3fn and
+    bfloat16 casts (round to nearest even) and at every midpoint between codes;
+    the scale exponent at exact powers 448 * 2^k and just above them; whole
+    tokens against the numpy/torch writer of the synthetic workloads; the
+    scatter against hand-computed (page, slot) offsets.
 """
 from __future__ import annotations
 
@@ -244,6 +249,111 @@ def check_combine_identity(lib=None):
     _close(co[0, 0], (math.e * a + bvec) / (math.e + 1.0), atol=1e-14)
 
 
+# ---------------------------------------------------------------- cache writer
+def check_e4m3_encode(lib=None):
+    # every finite code round-trips, both signs (0x80 is -0)
+    for c in list(range(0x7F)) + list(range(0x80, 0xFF)):
+        assert oracle.e4m3_encode(oracle.e4m3(c, lib), lib) == c, hex(c)
+    # the midpoint between two neighbouring codes goes to the even one; a hair either side to the nearer
+    for c in range(0x7E):
+        lo, hi = oracle.e4m3(c, lib), oracle.e4m3(c + 1, lib)
+        mid = 0.5 * (lo + hi)
+        assert oracle.e4m3_encode(mid, lib) == (c if c % 2 == 0 else c + 1), hex(c)
+        assert oracle.e4m3_encode(mid - (hi - lo) * 1e-6, lib) == c
+        assert oracle.e4m3_encode(mid + (hi - lo) * 1e-6, lib) == c + 1
+        assert oracle.e4m3_encode(-mid, lib) == 0x80 | (c if c % 2 == 0 else c + 1)
+    # saturation and special values
+    for x, code in ((448.0, 0x7E), (460.0, 0x7E), (1e6, 0x7E), (np.inf, 0x7E), (-np.inf, 0xFE), (-500.0, 0xFE),
+                    (np.nan, 0x7F), (0.0, 0x00), (-0.0, 0x80), (2.0 ** -11, 0x00), (3 * 2.0 ** -11, 0x01)):
+        assert oracle.e4m3_encode(x, lib) == code, (x, hex(oracle.e4m3_encode(x, lib)), hex(code))
+    # against torch's cast (round to nearest even) on float32 values inside the finite range
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal(4000) * np.exp2(rng.uniform(-14, 9, 4000))).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v), lib) for v in x], np.uint8)
+    assert np.array_equal(got, ref), np.flatnonzero(got != ref)[:5]
+
+
+def check_bf16_encode(lib=None):
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0, 1 << 32, 20000, dtype=np.uint64).astype(np.uint32)
+    bits = bits[((bits >> 23) & 0xFF) != 0xFF]  # finite binary32 values (subnormals included)
+    ties = (rng.integers(0, 1 << 16, 200, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000  # exact midpoints
+    ties = ties[((ties >> 23) & 0xFF) != 0xFF]
+    x = np.concatenate([bits, ties]).view(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.bf16_encode(float(v), lib) for v in x], np.uint16)
+    assert np.array_equal(got, ref), np.flatnonzero(got != ref)[:5]
+    assert oracle.bf16_encode(float("nan"), lib) == 0x7FC0
+    assert oracle.bf16_encode(float("inf"), lib) == 0x7F80 and oracle.bf16_encode(float("-inf"), lib) == 0xFF80
+    assert oracle.bf16_encode(3.4e38, lib) == 0x7F80  # past the largest finite bf16 by more than half an ulp
+
+
+def check_scale_exponent(lib=None):
+    g = np.zeros(64, np.float32)
+    assert oracle.scale_exponent(g, lib) == -127  # all zero
+    for k in (-120, -30, -8, -1, 0, 1, 5, 20, 100, 119):  # 448 * 2^119 is the largest in binary32
+        a = np.float32(448.0 * 2.0 ** k)
+        g[:] = 0.0
+        g[17] = -a
+        assert oracle.scale_exponent(g, lib) == k, k  # amax exactly 448 * 2^k: x / 2^k fits
+        g[17] = np.nextafter(a, np.float32(np.inf))
+        assert oracle.scale_exponent(g, lib) == k + 1, k  # just above: one more
+    g[:] = 1.0
+    assert oracle.scale_exponent(g, lib) == -8  # 1 <= 448 * 2^-8 = 1.75 but > 0.875
+    g[:] = np.float32(1e-44)
+    assert oracle.scale_exponent(g, lib) == -127  # below 448 * 2^-127: clamped
+    g[3] = np.inf
+    assert oracle.scale_exponent(g, lib) == 127
+    g[3] = np.nan
+    assert oracle.scale_exponent(g, lib) == 127
+
+
+def check_quantize_vs_generator(lib=None):
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((24, 512)).astype(np.float32)
+    x[3] *= 20.0  # an outlier row
+    x[5, :64] *= 1e-3  # groups of very different magnitudes
+    x[6, 64:128] = 0.0  # an all-zero group
+    x[7, 128:192] *= 1e4
+    rows, scales = W.quantize_rows(x)
+    for i in range(x.shape[0]):
+        r, sc = oracle.quantize_token(x[i], lib)
+        assert np.array_equal(r, rows[i]), i
+        assert np.array_equal(sc, scales[i]), i
+    # decoding a written token gives every nope value within half an e4m3 step of x / 2^e (times 2^e)
+    cache = np.zeros((1, W.PAGE_BYTES), np.uint8)
+    written = oracle.write_kv(x[:2], [0, 0], [5, 200], np.array([[0]], np.int32), cache, lib)
+    assert written == 0
+    lat, _ = oracle.gather(cache, np.array([[0]], np.int32), np.array([[5, 200]], np.int32),
+                           np.array([256], np.int32), lib)
+    for j in range(2):
+        for g in range(7):
+            e = oracle.scale_exponent(x[j, 64 * g:64 * g + 64], lib)
+            step = np.exp2(np.floor(np.log2(np.maximum(np.abs(x[j, 64 * g:64 * g + 64]) / 2.0 ** e, 2.0 ** -6))) - 3)
+            assert np.all(np.abs(lat[0, j, 64 * g:64 * g + 64] - x[j, 64 * g:64 * g + 64]) <= 0.5 * step * 2.0 ** e)
+
+
+def check_write_scatter(lib=None):
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((6, 512)).astype(np.float32)
+    bt = np.array([[2, 0], [1, -1]], np.int32)  # request 0: pages 2, 0; request 1: page 1, then none
+    cache = np.full((3, W.PAGE_BYTES), 0xA5, np.uint8)
+    req = np.array([0, 0, 1, 1, 2, 0], np.int32)
+    pos = np.array([3, 300, 255, 256, 0, -1], np.int32)  # (0,3) (0,300) (1,255) ok; the rest skipped
+    skipped = oracle.write_kv(x, req, pos, bt, cache, lib)
+    assert skipped == 3
+    expect = np.full((3, W.PAGE_BYTES), 0xA5, np.uint8)
+    for i, (page, slot) in enumerate([(2, 3), (0, 44), (1, 255)]):
+        r, sc = oracle.quantize_token(x[i], lib)
+        expect[page, slot * 576:(slot + 1) * 576] = r
+        expect[page, 147456 + slot * 8:147456 + slot * 8 + 8] = sc
+    assert np.array_equal(cache, expect)
+
+
 ALL_CHECKS = [check_e4m3, check_ue8m0, check_bf16, check_translation_fixture, check_byte_layout,
               check_two_token_closed_form, check_single_and_equal_slots, check_zero_q_mean,
-              check_permutation_and_padding, check_dense_brute_force, check_combine_identity]
+              check_permutation_and_padding, check_dense_brute_force, check_combine_identity,
+              check_e4m3_encode, check_bf16_encode, check_scale_exponent, check_quantize_vs_generator,
+              check_write_scatter]

@@ -36,6 +36,15 @@ MUTANTS = {
                              "qh[d] = orc_bf16(q[((int64_t)b * H + (H - 1 - h)) * ORC_DIM + d]);\n                orc_attend_one(qh, K, n, sm_scale, out + ((int64_t)b * H + h)"),
     "combine_weights_unnormalised": ("for (d = 0; d < ORC_DIM; d++) o[d] /= W;", ";"),
     "combine_lse_plain_max": ("lse[bh] = Lmax + log(W);", "lse[bh] = Lmax;"),
+    "encode_ties_to_odd": ("if (d < best_d || (d == best_d && (c & 1) == 0)) {", "if (d < best_d || (d == best_d && (c & 1) == 1)) {"),
+    "encode_sign_dropped": ("uint8_t sign = signbit(x) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
+    "bf16_truncates": ("    if (dlo < dhi) return lo;", "    if (dlo < dhi + 1.0) return lo;"),
+    "scale_exponent_floor": ("while (e < 127 && ldexp(448.0, e) < amax) e++;", "while (e < 127 && ldexp(448.0, e) <= amax) e++;"),
+    "scale_byte_bias": ("scale_row[g] = (uint8_t)(e + 127);", "scale_row[g] = (uint8_t)(e + 128);"),
+    "quantize_without_scale": ("row[d] = orc_e4m3_encode(ldexp((double)x[d], -e));", "row[d] = orc_e4m3_encode((double)x[d]);"),
+    "writer_rope_big_endian": ("row[ORC_NOPE + 2 * r] = (uint8_t)(u & 0xFF);", "row[ORC_NOPE + 2 * r] = (uint8_t)(u >> 8);"),
+    "writer_slot_from_block": ("page_base + (int64_t)(p % ORC_PAGE_TOKENS) * ORC_ROW_BYTES,", "page_base + (int64_t)(p / ORC_PAGE_TOKENS) * ORC_ROW_BYTES,"),
+    "writer_no_page_check": ("        if (page < 0 || (int64_t)page >= num_pages) {\n            skipped++;", "        if (page < -1000) {\n            skipped++;"),
 }
 
 
