@@ -190,6 +190,34 @@ int smla_decode_noalloc(const void *q, const uint8_t *kv_cache, const int32_t *b
                         const int32_t *seq_lens, float sm_scale, float *out, float *lse, int B, int H, int topk,
                         int max_blocks, int num_pages, void *stream);
 
+/*
+ * smla_write_kv -- the KV-cache writer: quantise n new latents into the cache format
+ * above and store each at position pos[i] of request req[i], i.e. at page
+ * block_table[req[i]][pos[i] / 256], slot pos[i] % 256 (the page indexing of "The
+ * Validation Moment"; the byte layout of "The Validation Gate", "The Test Design").
+ * The pages do not say how the scales are chosen; the rule here is that of the
+ * synthetic caches: per 64-dim nope group g, e = the smallest integer with
+ * max|x| <= 448 * 2^e, clamped to [-127, 127] (-127 for an all-zero group); scale
+ * byte g = e + 127 (byte 7 = 0); nope byte d = e4m3 of x[d] / 2^e, round to nearest
+ * even; rope value r = bf16 of x[448 + r], round to nearest even.  Non-finite
+ * inputs: a group holding an infinity or NaN takes e = 127, +-inf becomes +-448
+ * (0x7E / 0xFE) and NaN 0x7F; a NaN rope value becomes 0x7FC0.
+ *   latents     device, [n][512], fp32 (latents_bf16 = 0) or bf16 (latents_bf16 = 1),
+ *               16-byte aligned
+ *   req, pos    device, int32 [n]: request and position of each token
+ *   block_table device, int32 [B][max_blocks]
+ *   kv_cache    device, uint8 [num_pages][149504], 16-byte aligned (written)
+ *   err         device uint32 or NULL: SMLA_FLAG_BAD_PAGE is or-ed in when a token
+ *               is skipped (req outside [0, B), pos < 0, pos / 256 >= max_blocks, or
+ *               a page outside [0, num_pages)); nothing is written for it
+ *   n >= 0 (0: nothing is launched), B >= 1, max_blocks >= 1, 1 <= num_pages < 2^23.
+ * Two tokens with the same destination in one call: one of them is stored (which one
+ * is unspecified).  One launch on `stream`, one warp per token.
+ */
+int smla_write_kv(const void *latents, int latents_bf16, int n, const int32_t *req, const int32_t *pos,
+                  const int32_t *block_table, int B, int max_blocks, int num_pages, uint8_t *kv_cache,
+                  uint32_t *err, void *stream);
+
 /* Build identification string (static storage). */
 const char *smla_version(void);
 

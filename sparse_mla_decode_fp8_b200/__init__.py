@@ -21,4 +21,5 @@ from .binding import (  # noqa: F401
     read_error,
     version,
     workspace_bytes,
+    write_kv,
 )

@@ -67,6 +67,8 @@ def library():
             lib.smla_read_error.restype = I
             lib.smla_debug_gather.argtypes = [P, P, P, P, I, I, I, I, P, P, P, Z, P]
             lib.smla_debug_gather.restype = I
+            lib.smla_write_kv.argtypes = [P, I, I, P, P, P, I, I, I, P, P, P]
+            lib.smla_write_kv.restype = I
             lib.smla_version.restype = ctypes.c_char_p
             _lib = lib
     return _lib
@@ -176,3 +178,27 @@ def debug_gather(kv_cache, block_table, topk_idx, seq_lens, workspace=None, stre
         _stream(stream))
     _check(rc, "smla_debug_gather")
     return lat, ps
+
+
+def write_kv(latents, req, pos, block_table, kv_cache, err=None, stream=None) -> None:
+    """smla_write_kv: quantise latents [n,512] (fp32 or bf16) into ``kv_cache`` at position
+    pos[i] of request req[i]; ``err`` (a uint32 CUDA tensor of one element, or None)
+    receives SMLA_FLAG_BAD_PAGE when a token's destination is out of range."""
+    if latents.dtype not in (torch.float32, torch.bfloat16):
+        raise SmlaError("latents must be float32 or bfloat16")
+    n = latents.shape[0] if latents.dim() == 2 else 0
+    if latents.dim() != 2 or latents.shape[1] != DIM:
+        raise SmlaError("latents must be [n, 512]")
+    if req.shape != (n,) or pos.shape != (n,):
+        raise SmlaError("req and pos must be [n]")
+    ep = None
+    if err is not None:
+        if err.dtype not in (torch.int32, torch.uint32) or err.numel() < 1 or not err.is_cuda:
+            raise SmlaError("err must be a CUDA int32/uint32 tensor")
+        ep = err.data_ptr()
+    rc = library().smla_write_kv(
+        _dev(latents, latents.dtype, "latents"), 1 if latents.dtype == torch.bfloat16 else 0, n,
+        _dev(req, torch.int32, "req"), _dev(pos, torch.int32, "pos"), _dev(block_table, torch.int32, "block_table"),
+        block_table.shape[0], block_table.shape[1], kv_cache.shape[0], _dev(kv_cache, torch.uint8, "kv_cache"), ep,
+        _stream(stream))
+    _check(rc, "smla_write_kv")
