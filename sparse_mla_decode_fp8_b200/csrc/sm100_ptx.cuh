@@ -273,13 +273,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-// The upper 16 bits of two fp32 values as bf16x2 (truncation); `lo` goes to the low half.
-__device__ __forceinline__ uint32_t pack_bf16x2_trunc(float lo, float hi) {
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
-    return r;
-}
-
 // Two fp32 -> bf16x2 (round to nearest even); `lo` goes to the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

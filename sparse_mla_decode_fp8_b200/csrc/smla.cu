@@ -521,8 +521,8 @@ struct Worker {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float a0 = x[8 * half + 2 * e], a1 = x[8 * half + 2 * e + 1];
-                // hi = the top 16 bits of p (exact bf16), lo = bf16(p - hi): ~16 significant bits
-                hw[e] = pack_bf16x2_trunc(a0, a1);
+                // hi = bf16(p), lo = bf16(p - hi) (p - hi is exact in fp32): |p - hi - lo| <= 2^-17 p
+                hw[e] = pack_bf16x2(a0, a1);
                 lw[e] = pack_bf16x2(a0 - __uint_as_float(hw[e] << 16), a1 - __uint_as_float(hw[e] & 0xFFFF0000u));
             }
             const uint32_t off = r * 128 + (((2 * hq + half) ^ (r & 7)) << 4);
