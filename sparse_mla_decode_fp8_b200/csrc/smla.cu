@@ -213,9 +213,10 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volat
 // Warp-uniform version: lane 0 waits (acquire), the verdict is broadcast, and the warp
 // synchronisation orders the other lanes after its observation.
 __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                                const DecodeParams &p, int lane) {
+                                                const DecodeParams &p, int lane,
+                                                uint32_t backoff_ns = kWorkerBackoffNs) {
     int ok = 1;
-    if (lane == 0) ok = wait_phase(bar, parity, abort_flag, p, kWorkerBackoffNs) ? 1 : 0;
+    if (lane == 0) ok = wait_phase(bar, parity, abort_flag, p, backoff_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -229,10 +230,11 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
 // the barrier (every worker calls these with the same arguments).  Returns false if
 // the wait failed or was skipped.
 __device__ __forceinline__ bool workers_wait(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
-                                             bool enabled = true, uint32_t backoff_ns = kWorkerBackoffNs) {
+                                             bool enabled = true, uint32_t backoff_ns = kWorkerBackoffNs,
+                                             bool failed_before = false) {
     bool ok = enabled;
     if (t == kWaiter && enabled) ok = wait_phase(bar, parity, sm_abort(), p, backoff_ns);
-    return !barrier_or(kBarIdWorkers, kWorkers, !ok);
+    return !barrier_or(kBarIdWorkers, kWorkers, !ok || failed_before);
 }
 
 // ------------------------------------------------------------------ gather + dequant
@@ -338,13 +340,23 @@ __device__ __forceinline__ void publish_chunk(int c, int lane, uint64_t *bars) {
 // (`next`, null for the last tile): the load issue, which stalls while the memory
 // pipeline is full, overlaps the waits for the PV instead of delaying the softmax.
 __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const DecodeParams &p, Slot &s,
-                                             const int *next) {
+                                             const int *next, bool &late_ok) {
     const uint32_t kv = smem_addr(g_smem + kSmemKV);
     uint64_t *bars = sm_bars();
     const int k8 = t & 7;
+    // Chunk 0 waits as the whole worker group (its barrier also orders the previous step's
+    // writes of tile i+1's codes before every thread's loads below); chunks 1..3 wait warp
+    // by warp, so no warp waits for the slowest one of the chunk before.  A failed warp
+    // wait keeps the warp in step (it still stores and publishes) and is folded into the
+    // next worker-wide wait, where every worker sees it.
+    late_ok = true;
 #pragma unroll 1
     for (int c = 0; c < 3; ++c) {
-        if (i > 0 && !workers_wait(&bars[kBarKvFree + c], (i - 1) & 1, p, t)) return false;
+        if (c == 0) {
+            if (i > 0 && !workers_wait(&bars[kBarKvFree], (i - 1) & 1, p, t)) return false;
+        } else if (i > 0) {
+            late_ok = warp_wait_phase(&bars[kBarKvFree + c], (i - 1) & 1, sm_abort(), p, lane, 0u) && late_ok;
+        }
         const int kb = 2 * c + (k8 >> 2);  // also the scale group of these 16 dims
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -355,7 +367,7 @@ __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const Decod
         publish_chunk(c, lane, bars);
         if (next) load_part(c, t, next, p.cache, s);
     }
-    if (i > 0 && !workers_wait(&bars[kBarKvFree + 3], (i - 1) & 1, p, t)) return false;
+    if (i > 0) late_ok = warp_wait_phase(&bars[kBarKvFree + 3], (i - 1) & 1, sm_abort(), p, lane, 0u) && late_ok;
     store_item(kv, t >> 2, 6, 2 * (t & 3), true, s.nope3, s.sc3);
 #pragma unroll
     for (int u = 0; u < 2; ++u) store_item(kv, (t >> 3) + 64 * u, 7, k8, false, s.rope[u], 0u);
@@ -487,9 +499,9 @@ struct Worker {
     // kRescaleThreshold; P^T is written as bf16 hi + lo terms.  The scores are read from
     // tensor memory once; the running sums, which the PV does not read, are updated
     // after P^T has been handed to the tensor core.
-    __device__ __forceinline__ bool softmax(int i) {
+    __device__ __forceinline__ bool softmax(int i, bool failed_before = false) {
         // the tensor core is idle until P^T is written: wake up without backoff
-        if (!workers_wait(&sm_bars()[kBarSFull + (i & 1)], (i >> 1) & 1, p, t, true, 0u)) return false;
+        if (!workers_wait(&sm_bars()[kBarSFull + (i & 1)], (i >> 1) & 1, p, t, true, 0u, failed_before)) return false;
         tc_fence_after_sync();
         const float c = p.scale_log2;
         const bool valid = (sm_mask()[(i & 3) * 4 + q] >> lane) & 1u;
@@ -636,8 +648,9 @@ __device__ __forceinline__ bool worker_step(Worker &w, int i, int n, int t_begin
         tr.idx_b = (i + 3 < n && s3 < p.topk) ? __ldg(idx_row + s3) : -1;
     }
     const int *next = (i + 1 < n) ? sm_codes() + ((i + 1) & 1) * kTile : nullptr;
-    if (!dequant_tile(i, t, w.lane, p, cur, next)) return false;  // uniform over the workers
-    if (!w.softmax(i)) return false;
+    bool late_ok;
+    if (!dequant_tile(i, t, w.lane, p, cur, next, late_ok)) return false;  // uniform over the workers
+    if (!w.softmax(i, !late_ok)) return false;                           // uniform too
     if (t < kTile && i + 2 < n) {
         // tile i's codes are dead (its rows were loaded one step ago): tile i+2 takes the buffer
         const int code = slot_in_range(tr.idx_a, seq_len, p.max_blocks)
