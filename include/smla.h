@@ -38,9 +38,11 @@
  *   - Return value: SMLA_OK, or a negative SMLA_ERR_* code; on error nothing is
  *     launched.
  *   - Problems found on the device (a block-table entry outside [0,num_pages), a
- *     wait that ran out) do not fault: the affected token is masked or the CTA
- *     exits, and a bit is set in the sticky error word at the start of the
- *     workspace, read (and cleared) with smla_read_error.
+ *     wait that ran out) do not fault: the affected token is masked, or the CTA
+ *     gives up and writes NaN into its requests' rows of out and lse (so the result
+ *     is visibly invalid even if the error word is never read), and a bit is set in
+ *     the sticky error word at the start of the workspace, read (and cleared) with
+ *     smla_read_error.
  *   - Input domain: the cache holds no e4m3 NaN codes (0x7F/0xFF); dequantised
  *     nope values are exact in bf16 for scale bytes 10..254 as long as they lie
  *     in the bf16 range (larger ones become +-inf; scale bytes below 10 can round
@@ -65,7 +67,7 @@ extern "C" {
 
 /* Bits of the device error word. */
 #define SMLA_FLAG_BAD_PAGE 0x1u  /* a block-table entry outside [0, num_pages) was met and masked */
-#define SMLA_FLAG_TIMEOUT 0x2u   /* a pipeline wait ran out of time; that CTA wrote no output */
+#define SMLA_FLAG_TIMEOUT 0x2u   /* a pipeline wait ran out of time; that CTA's out/lse rows are NaN */
 #define SMLA_FLAG_SMEM 0x4u      /* dynamic shared memory was not 1024-byte aligned; CTA exited */
 
 #define SMLA_HEADS 64
@@ -104,12 +106,14 @@ typedef struct smla_options {
  *   workspace   device scratch of at least smla_workspace_bytes(B, H, topk)
  *               bytes, 256-byte aligned.  Its first 4 bytes are the sticky error
  *               word: zero it once (cudaMemset or smla_read_error) before first use.
- *               The rest holds the split-K exchange of a call (partials between
- *               the CTAs of a request, or between the decode and merge kernels);
+ *               The rest holds the split-K partials of a call that splits a request
+ *               in 3 or more parts (between the decode and the merge kernel);
  *               concurrent calls must not share a workspace.
  * Launches the decode kernel on `stream`.  A request whose topk range is split
- * in 2..4 parts is merged inside the kernel by the thread-block cluster of its
- * parts; with more parts the combine kernel follows.
+ * in 2 parts is merged inside the kernel by its CTA pair (one thread-block
+ * cluster: each adds its weighted part into out, two terms, so the result does
+ * not depend on their order); with 3 or more parts the combine kernel follows
+ * (a fixed summation order).  Results are reproducible bit for bit.
  */
 int smla_decode(const void *q, const uint8_t *kv_cache, const int32_t *block_table, const int32_t *topk_idx,
                 const int32_t *seq_lens, float sm_scale, float *out, float *lse, int B, int H, int topk,
