@@ -68,7 +68,7 @@ extern "C" {
 /* Bits of the device error word. */
 #define SMLA_FLAG_BAD_PAGE 0x1u  /* a block-table entry outside [0, num_pages) was met and masked */
 #define SMLA_FLAG_TIMEOUT 0x2u   /* a pipeline wait ran out of time; that CTA's out/lse rows are NaN */
-#define SMLA_FLAG_SMEM 0x4u      /* dynamic shared memory was not 1024-byte aligned; CTA exited */
+#define SMLA_FLAG_SMEM 0x4u      /* dynamic shared memory was not 1024-byte aligned; rows are NaN */
 
 #define SMLA_HEADS 64
 #define SMLA_DIM 512

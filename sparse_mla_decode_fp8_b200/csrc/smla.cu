@@ -327,16 +327,8 @@ __device__ __forceinline__ void store_item(uint32_t kv, int r, int kb, int oc, b
     }
 }
 
-// Publishes dims chunk c of the tile to the tensor core once this warp's stores are
-// visible to the async proxy.
-__device__ __forceinline__ void publish_chunk(int c, int lane, uint64_t *bars) {
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[kBarKvFull + c]);
-}
-
-// Dequantisation of tile i: each dims chunk is written as soon as the PV of tile i-1
-// has released it, and its registers then take the same chunk's rows of tile i+1
+// Dequantisation of tile i: each half of the dims is written as soon as the PV of tile
+// i-1 has released it, and its registers then take the same dims' rows of tile i+1
 // (`next`, null for the last tile): the load issue, which stalls while the memory
 // pipeline is full, overlaps the waits for the PV instead of delaying the softmax.
 __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const DecodeParams &p, Slot &s,
@@ -344,35 +336,58 @@ __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const Decod
     const uint32_t kv = smem_addr(g_smem + kSmemKV);
     uint64_t *bars = sm_bars();
     const int k8 = t & 7;
-    // Chunk 0 waits as the whole worker group (its barrier also orders the previous step's
-    // writes of tile i+1's codes before every thread's loads below); chunks 1..3 wait warp
-    // by warp, so no warp waits for the slowest one of the chunk before.  A failed warp
-    // wait keeps the warp in step (it still stores and publishes) and is folded into the
-    // next worker-wide wait, where every worker sees it.
+    // Two halves of 256 dims, each written in one go and published with one fence: half 0
+    // (dims chunks 0-1) after a worker-wide wait on chunk 1's release (the PV commits
+    // complete in issue order, so chunk 0 is free too; the barrier also orders the previous
+    // step's writes of tile i+1's codes before every thread's loads below), half 1 (chunks
+    // 2-3) after a warp-by-warp wait on chunk 3's.  A failed warp wait keeps the warp in
+    // step (it still stores and publishes) and is folded into the next worker-wide wait,
+    // where every worker sees it.  Fewer, larger hand-overs than one per 128-dim chunk: the
+    // waits, fences and arrivals cost more than the later start of the first half.
     late_ok = true;
-#pragma unroll 1
-    for (int c = 0; c < 3; ++c) {
-        if (c == 0) {
-            if (i > 0 && !workers_wait(&bars[kBarKvFree], (i - 1) & 1, p, t)) return false;
-        } else if (i > 0) {
-            late_ok = warp_wait_phase(&bars[kBarKvFree + c], (i - 1) & 1, sm_abort(), p, lane, 0u) && late_ok;
-        }
-        const int kb = 2 * c + (k8 >> 2);  // also the scale group of these 16 dims
+    if (i > 0 && !workers_wait(&bars[kBarKvFree + 1], (i - 1) & 1, p, t)) return false;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const int kb = 2 * c + (k8 >> 2);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const uint4 raw = (c == 0) ? s.raw[0][u] : (c == 1) ? s.raw[1][u] : s.raw[2][u];
+            const uint4 raw = (c == 0) ? s.raw[0][u] : s.raw[1][u];
             const uint32_t w = (kb < 4) ? s.srow[u].x : s.srow[u].y;
             store_item(kv, (t >> 3) + 64 * u, kb, 2 * (k8 & 3), true, raw, (w >> (8 * (kb & 3))) & 0xFFu);
         }
-        publish_chunk(c, lane, bars);
-        if (next) load_part(c, t, next, p.cache, s);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        mbar_arrive(&bars[kBarKvFull + 0]);
+        mbar_arrive(&bars[kBarKvFull + 1]);
+    }
+    if (next) {
+        load_part(0, t, next, p.cache, s);
+        load_part(1, t, next, p.cache, s);
     }
     if (i > 0) late_ok = warp_wait_phase(&bars[kBarKvFree + 3], (i - 1) & 1, sm_abort(), p, lane, 0u) && late_ok;
+    {
+        const int kb = 4 + (k8 >> 2);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint32_t w = (kb < 4) ? s.srow[u].x : s.srow[u].y;
+            store_item(kv, (t >> 3) + 64 * u, kb, 2 * (k8 & 3), true, s.raw[2][u], (w >> (8 * (kb & 3))) & 0xFFu);
+        }
+    }
     store_item(kv, t >> 2, 6, 2 * (t & 3), true, s.nope3, s.sc3);
 #pragma unroll
     for (int u = 0; u < 2; ++u) store_item(kv, (t >> 3) + 64 * u, 7, k8, false, s.rope[u], 0u);
-    publish_chunk(3, lane, bars);
-    if (next) load_part(3, t, next, p.cache, s);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        mbar_arrive(&bars[kBarKvFull + 2]);
+        mbar_arrive(&bars[kBarKvFull + 3]);
+    }
+    if (next) {
+        load_part(2, t, next, p.cache, s);
+        load_part(3, t, next, p.cache, s);
+    }
     return true;
 }
 
@@ -793,10 +808,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int split = blockIdx.x;
     const int b = blockIdx.y;
 
-    // The dynamic shared memory base is the same for every CTA of the launch, so this
-    // exit is uniform: no CTA of a cluster can be left waiting for a peer that took it.
+    // The shared-memory tiles need a 1024-byte aligned base (128-byte swizzle atoms).  The
+    // dynamic shared memory base is the same for every CTA of the launch, so this exit is
+    // taken by all CTAs or none.
     if (smem_addr(g_smem) & 1023u) {
         if (tid == 0) atomicOr(p.err, SMLA_FLAG_SMEM);
+        // the result is invalid: NaN where this CTA's output goes (the merge kernel turns a
+        // NaN partial log-sum-exp into NaN rows)
+        if (p.nsplit <= kMaxClusterSplits) {
+            float *o = p.out + static_cast<size_t>(b) * kHeads * kDim;
+            for (int k = tid; k < kHeads * kDim; k += kThreads) o[k] = NAN;
+            if (tid < kHeads) p.lse[static_cast<size_t>(b) * kHeads + tid] = NAN;
+        } else if (tid < kHeads) {
+            p.part_lse[(static_cast<size_t>(b) * kHeads + tid) * p.nsplit + split] = NAN;
+        }
+        // a CTA of a pair still takes part in both cluster barriers, so its peer (which
+        // takes this same exit: every CTA of a launch has the same shared-memory base)
+        // never waits on it
+        if (p.cluster_merge) {
+            cluster_arrive();
+            cluster_wait();
+            cluster_arrive();
+            cluster_wait();
+        }
         return;
     }
     uint64_t *bars = sm_bars();
