@@ -80,7 +80,7 @@ extern "C" {
 /* Tuning and test options for smla_decode_ex.  Zero-initialise for defaults. */
 typedef struct smla_options {
     int nsplit;                  /* topk splits per request; 0 = built-in heuristic */
-    int reserved0;
+    int out_bf16;                /* 0: out is fp32; 1: out is bf16 (see smla_decode_ex) */
     uint64_t wait_timeout_ns;    /* bound on every in-kernel wait; 0 = 1 s */
     uint32_t debug_flags;        /* test hooks, 0 in normal use (see SMLA_DEBUG_*) */
     uint32_t reserved1;
@@ -107,8 +107,8 @@ typedef struct smla_options {
  *               bytes, 256-byte aligned.  Its first 4 bytes are the sticky error
  *               word: zero it once (cudaMemset or smla_read_error) before first use.
  *               The rest holds the split-K partials of a call that splits a request
- *               in 3 or more parts (between the decode and the merge kernel);
- *               concurrent calls must not share a workspace.
+ *               (between the decode and the merge kernel: 3 or more parts, or a
+ *               bf16 output); concurrent calls must not share a workspace.
  * Launches the decode kernel on `stream`.  A request whose topk range is split
  * in 2 parts is merged inside the kernel by its CTA pair (one thread-block
  * cluster: each adds its weighted part into out, two terms, so the result does
@@ -120,9 +120,14 @@ int smla_decode(const void *q, const uint8_t *kv_cache, const int32_t *block_tab
                 int max_blocks, int num_pages, void *workspace, size_t workspace_bytes, void *stream);
 
 /* smla_decode with explicit options (opts may be NULL).  With opts->nsplit set,
- * the workspace must hold smla_workspace_bytes_ex(B, H, topk, opts->nsplit). */
+ * the workspace must hold smla_workspace_bytes_ex(B, H, topk, opts->nsplit).
+ * With opts->out_bf16 = 1, out is bf16 [B][H][512] (16-byte aligned): the fp32
+ * result rounded to nearest even (|dO| up to 2^-9 |O| more than the fp32 output;
+ * the pages give no bf16 tolerance), lse stays fp32.  A split request then merges
+ * through the merge kernel (fp32 partials, one bf16 rounding), never through
+ * atomic adds, so the result stays reproducible. */
 int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_table, const int32_t *topk_idx,
-                   const int32_t *seq_lens, float sm_scale, float *out, float *lse, int B, int H, int topk,
+                   const int32_t *seq_lens, float sm_scale, void *out, float *lse, int B, int H, int topk,
                    int max_blocks, int num_pages, void *workspace, size_t workspace_bytes,
                    const smla_options *opts, void *stream);
 
@@ -141,7 +146,8 @@ int smla_combine(const float *part_o, const float *part_lse, int nsplit, float *
 /* Number of topk splits smla_decode uses for (B, topk) on the current device. */
 int smla_num_splits(int B, int H, int topk);
 
-/* Workspace bytes smla_decode needs (header + split-K partials); 0 on bad sizes. */
+/* Workspace bytes smla_decode needs (header + split-K partials for any split count
+ * above 1, whatever the output type); 0 on bad sizes. */
 size_t smla_workspace_bytes(int B, int H, int topk);
 
 /* Workspace bytes for an explicit split count (1 <= nsplit <= ceil(topk/128)). */

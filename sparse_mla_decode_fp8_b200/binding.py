@@ -33,7 +33,7 @@ class SmlaError(RuntimeError):
 
 
 class _Options(ctypes.Structure):
-    _fields_ = [("nsplit", ctypes.c_int), ("reserved0", ctypes.c_int), ("wait_timeout_ns", ctypes.c_uint64),
+    _fields_ = [("nsplit", ctypes.c_int), ("out_bf16", ctypes.c_int), ("wait_timeout_ns", ctypes.c_uint64),
                 ("debug_flags", ctypes.c_uint32), ("reserved1", ctypes.c_uint32)]
 
 
@@ -120,21 +120,26 @@ def new_workspace(B: int, topk: int, nsplit: int = 0, device=None) -> torch.Tens
 
 
 def decode(q, kv_cache, block_table, topk_idx, seq_lens, sm_scale, out=None, lse=None, workspace=None,
-           nsplit: int = 0, wait_timeout_ns: int = 0, debug_flags: int = 0, stream=None):
-    """smla_decode_ex: returns (out fp32 [B,64,512], lse fp32 [B,64])."""
+           nsplit: int = 0, wait_timeout_ns: int = 0, debug_flags: int = 0, stream=None, out_dtype=None):
+    """smla_decode_ex: returns (out [B,64,512], lse fp32 [B,64]).  out is fp32, or bf16 when
+    ``out_dtype`` is torch.bfloat16 or a bf16 ``out`` tensor is given."""
     B, H, D = q.shape
     topk = topk_idx.shape[1]
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else torch.float32
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise SmlaError("out must be float32 or bfloat16")
     if out is None:
-        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+        out = torch.empty((B, H, D), dtype=out_dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = new_workspace(B, topk, nsplit, q.device)
-    opts = _Options(nsplit, 0, wait_timeout_ns, debug_flags, 0)
+    opts = _Options(nsplit, 1 if out_dtype == torch.bfloat16 else 0, wait_timeout_ns, debug_flags, 0)
     rc = library().smla_decode_ex(
         _dev(q, torch.bfloat16, "q"), _dev(kv_cache, torch.uint8, "kv_cache"),
         _dev(block_table, torch.int32, "block_table"), _dev(topk_idx, torch.int32, "topk_idx"),
-        _dev(seq_lens, torch.int32, "seq_lens"), float(sm_scale), _dev(out, torch.float32, "out"),
+        _dev(seq_lens, torch.int32, "seq_lens"), float(sm_scale), _dev(out, out_dtype, "out"),
         _dev(lse, torch.float32, "lse"), B, H, topk, block_table.shape[1], kv_cache.shape[0],
         _dev(workspace, torch.uint8, "workspace"), workspace.numel(), ctypes.byref(opts), _stream(stream))
     _check(rc, "smla_decode")

@@ -146,6 +146,7 @@ struct DecodeParams {
     float scale_log2;  // sm_scale * log2(e)
     uint32_t debug_flags;
     int cluster_merge;  // 1: the nsplit CTAs of a request form a cluster and merge in the kernel
+    int out_bf16;       // 1: out holds bf16 (written by this kernel with 1 split, else by the merge kernel)
 };
 
 // Reduces N (16 or 32) per-thread values across the 32 lanes of a warp, value i with
@@ -705,18 +706,29 @@ __device__ __forceinline__ void load_o16(uint32_t lane_addr, int c, int hq, floa
 // O^T, kChunkZero zeros (no tile, or weight 0), kChunkNan NaN (a failed wait: the result
 // is invalid).
 enum ChunkSource : int { kChunkNan = 0, kChunkZero = 1, kChunkTmem = 2 };
-__device__ __forceinline__ void write_chunk(const Worker &w, int c, const float (&scale)[16], float *dst,
-                                            size_t head_stride, int source, bool add) {
+__device__ __forceinline__ uint16_t to_bf16_rn(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+// kMode: kStoreF32 plain fp32 stores, kAddF32 atomic adds, kStoreBf16 bf16 stores.
+enum StoreMode : int { kStoreF32 = 0, kAddF32 = 1, kStoreBf16 = 2 };
+template <int kMode>
+__device__ __forceinline__ void write_chunk(const Worker &w, int c, const float (&scale)[16], void *dst,
+                                            size_t head_stride, int source) {
     float v[16];
     if (source == kChunkTmem) load_o16(w.tmem + w.lane_base, c, w.hq, v);
-    float *o = dst + static_cast<size_t>(16 * w.hq) * head_stride + 128 * c + 32 * w.q + w.lane;
+    const size_t off = static_cast<size_t>(16 * w.hq) * head_stride + 128 * c + 32 * w.q + w.lane;
 #pragma unroll
     for (int h = 0; h < 16; ++h) {
         const float x = (source == kChunkTmem) ? v[h] * scale[h] : (source == kChunkZero) ? 0.0f : NAN;
-        if (add)
-            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(o + h * head_stride), "f"(x) : "memory");
+        if (kMode == kStoreBf16)
+            static_cast<uint16_t *>(dst)[off + h * head_stride] = to_bf16_rn(x);
+        else if (kMode == kAddF32)
+            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(static_cast<float *>(dst) + off + h * head_stride), "f"(x)
+                         : "memory");
         else
-            o[h * head_stride] = x;
+            static_cast<float *>(dst)[off + h * head_stride] = x;
     }
 }
 
@@ -734,15 +746,23 @@ __device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int
         inv[w.t] = !ok ? NAN : (l > 0.0f) ? 1.0f / l : 0.0f;
     }
     named_barrier_sync(kBarIdWorkers, kWorkers);
-    // the nsplit > 1 partials are [b][head][split][dim]
+    // the nsplit > 1 partials are [b][head][split][dim] fp32; one split writes out (fp32 or bf16)
     const size_t head_stride = static_cast<size_t>(p.nsplit) * kDim;
-    float *base = (p.nsplit == 1) ? p.out + static_cast<size_t>(b) * kHeads * kDim
-                                  : p.part_o + static_cast<size_t>(b) * kHeads * head_stride + split * kDim;
+    const bool bf16 = p.nsplit == 1 && p.out_bf16;
+    void *base = (p.nsplit > 1) ? static_cast<void *>(p.part_o + static_cast<size_t>(b) * kHeads * head_stride +
+                                                      split * kDim)
+                 : bf16 ? static_cast<void *>(reinterpret_cast<uint16_t *>(p.out) + static_cast<size_t>(b) * kHeads * kDim)
+                        : static_cast<void *>(p.out + static_cast<size_t>(b) * kHeads * kDim);
     float sc[16];
     load16(inv + 16 * w.hq, sc);
     const int source = !ok ? kChunkNan : (n > 0) ? kChunkTmem : kChunkZero;
+    if (bf16) {
 #pragma unroll 1
-    for (int mc = 0; mc < 4; ++mc) write_chunk(w, mc, sc, base, head_stride, source, false);
+        for (int mc = 0; mc < 4; ++mc) write_chunk<kStoreBf16>(w, mc, sc, base, head_stride, source);
+    } else {
+#pragma unroll 1
+        for (int mc = 0; mc < 4; ++mc) write_chunk<kStoreF32>(w, mc, sc, base, head_stride, source);
+    }
 }
 
 // nsplit = 2 in one cluster.  With lambda_s = m_s + log2 l_s (the log-sum-exp of split s
@@ -790,7 +810,7 @@ __device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) 
         const bool chunk_ok = workers_wait(&bars[kBarKvFree + c], (n - 1) & 1, p, t, ok && n > 0);
         // a split without tiles adds zeros; a failed wait NaN
         const int source = chunk_ok ? kChunkTmem : (ok && n == 0) ? kChunkZero : kChunkNan;
-        write_chunk(w, c, sc, base, kDim, source, true);
+        write_chunk<kAddF32>(w, c, sc, base, kDim, source);
     }
 }
 
@@ -815,9 +835,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) atomicOr(p.err, SMLA_FLAG_SMEM);
         // the result is invalid: NaN where this CTA's output goes (the merge kernel turns a
         // NaN partial log-sum-exp into NaN rows)
-        if (p.nsplit <= kMaxClusterSplits) {
-            float *o = p.out + static_cast<size_t>(b) * kHeads * kDim;
-            for (int k = tid; k < kHeads * kDim; k += kThreads) o[k] = NAN;
+        if (p.cluster_merge || p.nsplit == 1) {
+            for (int k = tid; k < kHeads * kDim; k += kThreads) {
+                if (p.out_bf16)
+                    reinterpret_cast<uint16_t *>(p.out)[static_cast<size_t>(b) * kHeads * kDim + k] = 0x7FC0u;
+                else
+                    p.out[static_cast<size_t>(b) * kHeads * kDim + k] = NAN;
+            }
             if (tid < kHeads) p.lse[static_cast<size_t>(b) * kHeads + tid] = NAN;
         } else if (tid < kHeads) {
             p.part_lse[(static_cast<size_t>(b) * kHeads + tid) * p.nsplit + split] = NAN;
@@ -937,9 +961,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Split-K merge: one CTA of 128 threads per (b, h), 4 output dims per thread.
+__device__ __forceinline__ void store_row4(void *out, size_t bh, int tid, float4 v, int out_bf16) {
+    if (out_bf16) {
+        const uint32_t lo = to_bf16_rn(v.x) | (static_cast<uint32_t>(to_bf16_rn(v.y)) << 16);
+        const uint32_t hi = to_bf16_rn(v.z) | (static_cast<uint32_t>(to_bf16_rn(v.w)) << 16);
+        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(out) + bh * kDim)[tid] = make_uint2(lo, hi);
+    } else {
+        reinterpret_cast<float4 *>(static_cast<float *>(out) + bh * kDim)[tid] = v;
+    }
+}
+
 __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ part_o,
-                                                      const float *__restrict__ part_lse, float *__restrict__ out,
-                                                      float *__restrict__ lse, int nsplit) {
+                                                      const float *__restrict__ part_lse, void *__restrict__ out,
+                                                      float *__restrict__ lse, int nsplit, int out_bf16) {
     const size_t bh = blockIdx.x;
     const int tid = threadIdx.x;
     const float *L = part_lse + bh * nsplit;
@@ -952,12 +986,12 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
     }
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (invalid) {
-        reinterpret_cast<float4 *>(out + bh * kDim)[tid] = make_float4(NAN, NAN, NAN, NAN);
+        store_row4(out, bh, tid, make_float4(NAN, NAN, NAN, NAN), out_bf16);
         if (tid == 0) lse[bh] = NAN;
         return;
     }
     if (lmax == -INFINITY) {
-        reinterpret_cast<float4 *>(out + bh * kDim)[tid] = acc;
+        store_row4(out, bh, tid, acc, out_bf16);
         if (tid == 0) lse[bh] = -INFINITY;
         return;
     }
@@ -978,7 +1012,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float *__restrict__ 
     acc.y *= inv;
     acc.z *= inv;
     acc.w *= inv;
-    reinterpret_cast<float4 *>(out + bh * kDim)[tid] = acc;
+    store_row4(out, bh, tid, acc, out_bf16);
     if (tid == 0) lse[bh] = lmax + logf(wsum);
 }
 
@@ -1126,14 +1160,14 @@ bool sizes_ok(int B, int H, int topk) {
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Two splits of a request merge inside the decode kernel (a CTA pair: the log-sum-exp
-// rows cross through distributed shared memory, the outputs are added into out); more
-// go through normalised global partials and the merge kernel.
+// rows cross through distributed shared memory, the fp32 outputs are added into out);
+// more, or a bf16 output, go through normalised global partials and the merge kernel.
 //
-// Workspace after the header: nsplit <= 2: nothing.  Above 2: part_lse [B][64][nsplit]
-// f32, then part_o [B][64][nsplit][512] f32.
+// Workspace after the header: nsplit == 1: nothing.  nsplit >= 2: part_lse [B][64][nsplit]
+// f32, then part_o [B][64][nsplit][512] f32 (unused by the fp32 pair merge).
 size_t workspace_for(int B, int topk, int nsplit) {
     size_t bytes = SMLA_WORKSPACE_HEADER;
-    if (nsplit > smla::kMaxClusterSplits) {
+    if (nsplit > 1) {
         const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
         bytes += round256(rows * sizeof(float)) + rows * SMLA_DIM * sizeof(float);
     }
@@ -1177,12 +1211,12 @@ int smla_combine(const float *part_o, const float *part_lse, int nsplit, float *
     if (rc != SMLA_OK) return rc;
     (void)cudaGetLastError();
     smla::combine_kernel<<<static_cast<unsigned>(B) * static_cast<unsigned>(H), 128, 0,
-                           static_cast<cudaStream_t>(stream)>>>(part_o, part_lse, out, lse, nsplit);
+                           static_cast<cudaStream_t>(stream)>>>(part_o, part_lse, out, lse, nsplit, 0);
     return cudaGetLastError() == cudaSuccess ? SMLA_OK : SMLA_ERR_LAUNCH;
 }
 
 int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_table, const int32_t *topk_idx,
-                   const int32_t *seq_lens, float sm_scale, float *out, float *lse, int B, int H, int topk,
+                   const int32_t *seq_lens, float sm_scale, void *out, float *lse, int B, int H, int topk,
                    int max_blocks, int num_pages, void *workspace, size_t workspace_bytes,
                    const smla_options *opts, void *stream) {
     if (!q || !kv_cache || !block_table || !topk_idx || !seq_lens || !out || !lse || !workspace)
@@ -1206,11 +1240,12 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     p.block_table = block_table;
     p.topk_idx = topk_idx;
     p.seq_lens = seq_lens;
-    p.out = out;
+    p.out = static_cast<float *>(out);
+    p.out_bf16 = (opts && opts->out_bf16) ? 1 : 0;
     p.lse = lse;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.err = reinterpret_cast<uint32_t *>(ws);
-    if (nsplit > smla::kMaxClusterSplits) {
+    if (nsplit > 1) {
         const size_t rows = static_cast<size_t>(B) * SMLA_HEADS * nsplit;
         p.part_lse = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER);
         p.part_o = reinterpret_cast<float *>(ws + SMLA_WORKSPACE_HEADER + round256(rows * sizeof(float)));
@@ -1230,7 +1265,7 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     (void)cudaGetLastError();
-    p.cluster_merge = (nsplit > 1 && nsplit <= smla::kMaxClusterSplits) ? 1 : 0;
+    p.cluster_merge = (nsplit > 1 && nsplit <= smla::kMaxClusterSplits && !p.out_bf16) ? 1 : 0;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(nsplit, B);
     cfg.blockDim = dim3(smla::kThreads);
@@ -1247,7 +1282,7 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_LAUNCH;
     if (nsplit > 1 && !p.cluster_merge) {
         smla::combine_kernel<<<static_cast<unsigned>(B) * SMLA_HEADS, 128, 0, st>>>(p.part_o, p.part_lse, out, lse,
-                                                                                   nsplit);
+                                                                                   nsplit, p.out_bf16);
         if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_LAUNCH;
     }
     return SMLA_OK;

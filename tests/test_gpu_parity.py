@@ -108,6 +108,31 @@ def test_validation_matrix(B, topk, ragged):
     print(f"B={B} topk={topk} len={ragged}: nsplit={smla.num_splits(B, topk)} {figs}")
 
 
+# bf16 output (smla_options.out_bf16): the fp32 result rounded to nearest even, so the
+# bound is the fp32 one plus the rounding, 2^-9 |O| (2^-8 here for margin); LSE stays fp32.
+@pytest.mark.parametrize("k,ns", [(1, 0), (2, 0), (3, 0), (4, 0), (5, 0), (4, 1), (2, 2)])
+def test_bf16_output(k, ns):
+    w = W.make_config(k)
+    d = device_inputs(w)
+    args = (d["q"], d["kv_cache"], d["block_table"], d["topk_idx"], d["seq_lens"], d["sm_scale"])
+    out, lse = smla.decode(*args, nsplit=ns, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert out.dtype == torch.bfloat16 and lse.dtype == torch.float32
+    ro, rl = _oracle(w)
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    assert np.all(np.isfinite(o))
+    assert np.all(np.abs(o - ro) <= 2e-3 + 2.0 ** -8 * np.abs(ro))
+    assert np.linalg.norm(o - ro) <= 5e-3 * np.linalg.norm(ro)
+    fin = np.isfinite(rl)
+    assert np.array_equal(np.isneginf(l), np.isneginf(rl))
+    assert np.abs(l[fin] - rl[fin]).max() <= 1e-3
+    if (ns or smla.num_splits(w.B, w.topk)) == 1:
+        # one split: exactly the fp32 output rounded to nearest even, the same LSE
+        o32, l32 = smla.decode(*args, nsplit=ns)
+        assert torch.equal(out, o32.to(torch.bfloat16)) and torch.equal(lse, l32)
+
+
 @pytest.mark.parametrize("nsplit", [1, 2, 3, 4])
 def test_split_counts_agree(nsplit):
     w = W.make_config(2)
