@@ -454,9 +454,9 @@ def run_cuda(args):
     ms_step = max_ms / steps
     units = W.roofline_units(w.replica(0))
     peaks, peak_src = load_peaks()
-    # up to kMaxClusterSplits splits merge inside the decode kernel's cluster: one launch per call;
-    # beyond that a second (combine) kernel follows
-    launches_per_call = 1 if nsplit <= 4 else 2
+    # a request in 2 splits merges inside the decode kernel (the CTA pair's fp32 adds): one launch
+    # per call; 3 or more splits are merged by a second (combine) kernel
+    launches_per_call = 1 if nsplit <= 2 else 2
     # this rank's own average duration of one decode launch over the timed region (graph replays on `stream`)
     call_ms = elapsed_ms / steps
     achieved_gbs = units["bytes"] / (call_ms * 1e-3) / 1e9
