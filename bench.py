@@ -525,14 +525,40 @@ def _profiled_traffic(k: int):
     return int(fields["dram_bytes_per_launch"])
 
 
+def _code_tokens(src: str) -> str:
+    """The source with its comments removed and whitespace collapsed: what the compiler sees."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def _kernel_hash() -> str:
+    """Hash of the CUDA sources' code (comments and layout excluded), named in the ncu summaries."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_mla_decode_fp8_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+    files = [os.path.join(csrc, name) for name in sorted(os.listdir(csrc))]
+    for path in files + [os.path.join(ROOT, "include", "smla.h")]:
+        with open(path, encoding="utf-8") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + _code_tokens(f.read()).encode() + b"\0")
     return h.hexdigest()[:16]
 
 

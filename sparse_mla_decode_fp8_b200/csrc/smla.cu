@@ -10,28 +10,30 @@
 // their log-sum-exp (Step 5).
 //
 // B200 mapping, per CTA (one per SM, 16 worker warps + 1 control warp):
-//   * Q[b] (64 heads x 512, bf16) sits in shared memory (one TMA load) until the
-//     last score MMA; then that buffer receives the split merge's partials.
+//   * Q[b] (64 heads x 512, bf16) sits in shared memory (one TMA load) for the
+//     whole kernel: every tile's score MMA reads it there.
 //   * The worker warps hold the FP8 rows of the next 128-slot tile in registers
 //     (16-byte loads) while the rows of the tile after it are already on their
-//     way into L2 (bulk prefetches issued two tiles ahead), and dequantise a tile into a bf16 [128 x 512] buffer in the
-//     128-byte-swizzled layout the tensor core reads, one 128-dim chunk at a time
-//     as the previous tile's PV releases it.
+//     way into L2 (bulk prefetches issued two tiles ahead), and dequantise a tile
+//     into a bf16 [128 x 512] buffer in the 128-byte-swizzled layout the tensor
+//     core reads, in two 256-dim halves as the previous tile's PV releases them.
 //   * S^T[128 tokens x 64 heads] = K_tile . Q^T: tcgen05.mma M=128 N=64, fp32 in
 //     tensor memory.  Tokens fill the 128-row M dimension, not the 64 heads.
 //   * The worker warps then read S^T from tensor memory (one token lane and 16
-//     heads per thread), keep the running max per head, rescale O^T in tensor
-//     memory when the max grows, and write P^T as two bf16 terms (P = P_hi + P_lo).
-//   * O^T[512 x 64] += V^T . P^T with V = the same bf16 tile read MN-major: 4 MMAs
-//     of M=128 per 16-token step, once with P_hi and once with P_lo, so P carries
-//     ~16 significant bits (a single bf16 P is not accurate enough when a few
-//     large latents dominate).
+//     heads per thread), raise the running max of a head only when a score passes
+//     it by more than kRescaleThreshold (then O^T and the sums are rescaled in
+//     tensor memory), and write P^T as two bf16 terms (P = P_hi + P_lo).
+//   * O^T[512 x 64] += V^T . P^T with V = the same bf16 tile read MN-major: per
+//     16-token step, dims chunks 0-1 take one N=128 MMA each over [P_hi | P_lo],
+//     chunks 2-3 two N=64 MMAs each, so P carries ~16 significant bits (a single
+//     bf16 P is not accurate enough when a few large latents dominate).
 //   * The control warp owns tensor memory and the mbarriers, loads Q and issues
 //     every MMA from one thread.
-//   * The epilogue writes O/l and LSE = (m + log2 l) ln 2, or, when the topk range
-//     of a request is split over a thread-block cluster, streams each CTA's O^T
-//     through distributed shared memory to the CTA that owns those output dims as
-//     soon as the last PV has finished that chunk.
+//   * The epilogue writes O/l and LSE = (m + log2 l) ln 2.  When the topk range of
+//     a request is split in two, the two CTAs of a cluster swap their per-head
+//     log-sum-exps and each adds its scaled O^T into the output (zeroed half by
+//     each at entry) with fp32 atomic adds straight from tensor memory; more
+//     splits, or a bf16 output, write fp32 partials that combine_kernel merges.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -76,9 +78,11 @@ constexpr int kSmemBars = kSmemPeerLam + 256;     // mbarriers (8 B each)
 
 enum Bar : int {
     kBarQ = 0,          // Q landed (TMA transaction bytes)
-    kBarKvFull = 1,     // + c (c = 0..3): dims chunk c of the tile written (16 worker-warp arrivals)
+    kBarKvFull = 1,     // + c (c = 0..3): dims chunk c of the tile written (16 worker-warp arrivals;
+                        //   chunks 0-1 with the first 256-dim half, 2-3 with the second)
     kBarKvFree = 5,     // + c: PV chunk c of the tile done (MMA commit): chunk c may be overwritten
-    kBarSFull = 9,      // + s (s = 0..1): S^T buffer s complete (MMA commit)
+    kBarSFull = 9,      // + (i & 1): S^T of tile i complete (MMA commit; the two barriers alternate
+                        //   over the tiles, each completing once every second tile)
     kBarPFull = 11,     // P^T written (16 worker-warp arrivals)
     kBarDrain = 12,     // final commit before tensor memory is released
     kBarSpare = 13,     // test hook target
