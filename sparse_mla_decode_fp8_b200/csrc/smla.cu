@@ -149,9 +149,14 @@ struct DecodeParams {
     int tiles_per_split;
     float scale_log2;  // sm_scale * log2(e)
     uint32_t debug_flags;
-    int cluster_merge;  // 1: the nsplit CTAs of a request form a cluster and merge in the kernel
-    int out_bf16;       // 1: out holds bf16 (written by this kernel with 1 split, else by the merge kernel)
 };
+
+// What the decode kernel writes, fixed at compile time so each instantiation carries only
+// its own epilogue (and gets its own register allocation):
+//   kEpiF32   fp32 O and LSE with one split; fp32 partials for the merge kernel with more
+//   kEpiBf16  bf16 O (round to nearest even) and fp32 LSE, one split
+//   kEpiPair  two splits in a CTA pair (cluster) adding into the fp32 output
+enum Epilogue : int { kEpiF32 = 0, kEpiBf16 = 1, kEpiPair = 2 };
 
 // Reduces N (16 or 32) per-thread values across the 32 lanes of a warp, value i with
 // value i of every other lane.  Each round halves the live entries: a lane keeps the
@@ -736,6 +741,7 @@ __device__ __forceinline__ void write_chunk(const Worker &w, int c, const float 
     }
 }
 
+template <int kEpi>
 __device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int n, bool ok) {
     const DecodeParams &p = w.p;
     if (n > 0) ok = workers_wait(&sm_bars()[kBarKvFree + 3], (n - 1) & 1, p, w.t, ok);
@@ -752,7 +758,7 @@ __device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int
     named_barrier_sync(kBarIdWorkers, kWorkers);
     // the nsplit > 1 partials are [b][head][split][dim] fp32; one split writes out (fp32 or bf16)
     const size_t head_stride = static_cast<size_t>(p.nsplit) * kDim;
-    const bool bf16 = p.nsplit == 1 && p.out_bf16;
+    constexpr bool bf16 = kEpi == kEpiBf16;
     void *base = (p.nsplit > 1) ? static_cast<void *>(p.part_o + static_cast<size_t>(b) * kHeads * head_stride +
                                                       split * kDim)
                  : bf16 ? static_cast<void *>(reinterpret_cast<uint16_t *>(p.out) + static_cast<size_t>(b) * kHeads * kDim)
@@ -760,7 +766,7 @@ __device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int
     float sc[16];
     load16(inv + 16 * w.hq, sc);
     const int source = !ok ? kChunkNan : (n > 0) ? kChunkTmem : kChunkZero;
-    if (bf16) {
+    if constexpr (bf16) {
 #pragma unroll 1
         for (int mc = 0; mc < 4; ++mc) write_chunk<kStoreBf16>(w, mc, sc, base, head_stride, source);
     } else {
@@ -824,8 +830,10 @@ __device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) 
 // flight; the control warp issues the MMAs (S^T of tile i as its dims chunks land,
 // PV of tile i once P^T is written, each PV chunk releasing that chunk of the tile
 // buffer to the next tile's dequantisation).
+template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_q) {
+    constexpr bool kPair = kEpi == kEpiPair;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -839,9 +847,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) atomicOr(p.err, SMLA_FLAG_SMEM);
         // the result is invalid: NaN where this CTA's output goes (the merge kernel turns a
         // NaN partial log-sum-exp into NaN rows)
-        if (p.cluster_merge || p.nsplit == 1) {
+        if (kPair || p.nsplit == 1) {
             for (int k = tid; k < kHeads * kDim; k += kThreads) {
-                if (p.out_bf16)
+                if (kEpi == kEpiBf16)
                     reinterpret_cast<uint16_t *>(p.out)[static_cast<size_t>(b) * kHeads * kDim + k] = 0x7FC0u;
                 else
                     p.out[static_cast<size_t>(b) * kHeads * kDim + k] = NAN;
@@ -853,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a CTA of a pair still takes part in both cluster barriers, so its peer (which
         // takes this same exit: every CTA of a launch has the same shared-memory base)
         // never waits on it
-        if (p.cluster_merge) {
+        if constexpr (kPair) {
             cluster_arrive();
             cluster_wait();
             cluster_arrive();
@@ -892,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars[kBarSpare], 1);
             mbar_init(&bars[kBarMl], 1);
             // the peer's row of 64 log-sum-exps arrives as 256 transaction bytes
-            if (p.cluster_merge) mbar_arrive_expect_tx(&bars[kBarMl], kHeads * 4);
+            if (kPair) mbar_arrive_expect_tx(&bars[kBarMl], kHeads * 4);
             fence_barrier_init();
             *sm_abort() = 0;
             mbar_arrive_expect_tx(&bars[kBarQ], kHeads * kDim * 2);
@@ -915,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (tid < kHeads) head_m[tid] = -INFINITY;
-    if (p.cluster_merge) {
+    if constexpr (kPair) {
         // two splits add their weighted partials into the output: each CTA zeroes 32 heads of
         // out[b] now; the barriers below order these stores before either CTA's additions
         float4 *z = reinterpret_cast<float4 *>(p.out + (static_cast<size_t>(b) * kHeads + 32 * split) * kDim);
@@ -924,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (p.cluster_merge) cluster_arrive();  // peers may address this CTA's mbarriers from now on
+    if constexpr (kPair) cluster_arrive();  // peers may address this CTA's mbarriers from now on
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
 
@@ -932,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================================ MMA issue
         if (lane == 0 && n > 0) mma_issue_loop(tmem, p, n);
         __syncwarp();
-        if (p.cluster_merge) cluster_wait();
+        if constexpr (kPair) cluster_wait();
     } else {
         // ================================================================ workers
         Worker w{p, tmem, tid, warp, lane, warp & 3, warp >> 2, static_cast<uint32_t>(32 * (warp & 3)) << 16};
@@ -944,16 +952,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = ok && !*sm_abort();
         ok = !barrier_or(kBarIdWorkers, kWorkers, !ok);
         w.reduce_sums(ok && n > 0);
-        if (p.cluster_merge) {
+        if constexpr (kPair) {
             cluster_wait();  // the peer has initialised its mbarriers and zeroed its half of out
             epilogue_pair(w, b, n, ok);
         } else {
-            epilogue_direct(w, b, split, n, ok);
+            epilogue_direct<kEpi>(w, b, split, n, ok);
         }
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (p.cluster_merge) {
+    if constexpr (kPair) {
         // no CTA leaves while a peer may still write into its shared memory
         cluster_arrive();
         cluster_wait();
@@ -1132,8 +1140,12 @@ int device_info(DeviceInfo *&info) {
         d.supported = (major == 10 && minor == 0);
         d.sms = sms;
         if (d.supported &&
-            cudaFuncSetAttribute(smla::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smla::kSmemBytes) != cudaSuccess)
+            (cudaFuncSetAttribute(smla::decode_kernel<smla::kEpiF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smla::kSmemBytes) != cudaSuccess ||
+             cudaFuncSetAttribute(smla::decode_kernel<smla::kEpiBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smla::kSmemBytes) != cudaSuccess ||
+             cudaFuncSetAttribute(smla::decode_kernel<smla::kEpiPair>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smla::kSmemBytes) != cudaSuccess))
             return SMLA_ERR_CUDA;
         d.ready = true;
     }
@@ -1245,7 +1257,7 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     p.topk_idx = topk_idx;
     p.seq_lens = seq_lens;
     p.out = static_cast<float *>(out);
-    p.out_bf16 = (opts && opts->out_bf16) ? 1 : 0;
+    const bool out_bf16 = opts && opts->out_bf16;
     p.lse = lse;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.err = reinterpret_cast<uint32_t *>(ws);
@@ -1269,7 +1281,10 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     (void)cudaGetLastError();
-    p.cluster_merge = (nsplit > 1 && nsplit <= smla::kMaxClusterSplits && !p.out_bf16) ? 1 : 0;
+    // two splits merge inside the kernel (fp32 output); more, or a bf16 output with splits,
+    // go through fp32 partials and the merge kernel
+    const bool pair = nsplit > 1 && nsplit <= smla::kMaxClusterSplits && !out_bf16;
+    const int epi = pair ? smla::kEpiPair : (out_bf16 && nsplit == 1) ? smla::kEpiBf16 : smla::kEpiF32;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(nsplit, B);
     cfg.blockDim = dim3(smla::kThreads);
@@ -1277,16 +1292,20 @@ int smla_decode_ex(const void *q, const uint8_t *kv_cache, const int32_t *block_
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.cluster_merge ? nsplit : 1;
+    attr[0].val.clusterDim.x = pair ? nsplit : 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, smla::decode_kernel, p, tmap_q) != cudaSuccess) return SMLA_ERR_LAUNCH;
+    const cudaError_t launched =
+        epi == smla::kEpiPair   ? cudaLaunchKernelEx(&cfg, smla::decode_kernel<smla::kEpiPair>, p, tmap_q)
+        : epi == smla::kEpiBf16 ? cudaLaunchKernelEx(&cfg, smla::decode_kernel<smla::kEpiBf16>, p, tmap_q)
+                                : cudaLaunchKernelEx(&cfg, smla::decode_kernel<smla::kEpiF32>, p, tmap_q);
+    if (launched != cudaSuccess) return SMLA_ERR_LAUNCH;
     if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_LAUNCH;
-    if (nsplit > 1 && !p.cluster_merge) {
+    if (nsplit > 1 && !pair) {
         smla::combine_kernel<<<static_cast<unsigned>(B) * SMLA_HEADS, 128, 0, st>>>(p.part_o, p.part_lse, out, lse,
-                                                                                   nsplit, p.out_bf16);
+                                                                                   nsplit, out_bf16 ? 1 : 0);
         if (cudaGetLastError() != cudaSuccess) return SMLA_ERR_LAUNCH;
     }
     return SMLA_OK;

@@ -84,8 +84,9 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_shifted(uint32_t two_bytes)
 }
 
 // Scale bytes above 142: 2^(s-15) is not a bf16 normal, so multiply by 2^127 and then by
-// 2^(s-142); 0xFF gives NaN.  Out of line: such scales do not occur in normal caches.
-static __device__ __noinline__ void scale_big(uint32_t (&o)[8], uint32_t s) {
+// 2^(s-142); 0xFF gives NaN.  Inline like the common path: an out-of-line call would take
+// the address of o, which then lives in local memory on every dequantisation.
+__device__ __forceinline__ void scale_big(uint32_t (&o)[8], uint32_t s) {
     const uint32_t big = 0x7F007F00u;                              // 2^127 in both halves
     const uint32_t m = (s == 255u) ? 0x7FC0u : ((s - 15u) << 7);  // 2^(s-142) or NaN
     const uint32_t m2 = m | (m << 16);
