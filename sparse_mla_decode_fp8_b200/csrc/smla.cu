@@ -197,8 +197,8 @@ __device__ __forceinline__ void load16(const float *src, float (&v)[16]) {
 
 // Bounded wait on an mbarrier phase.  Gives up when another thread has aborted the
 // CTA or when `timeout_ns` passes (then it aborts the CTA and flags the error).
-__device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             const DecodeParams &p, uint32_t backoff_ns) {
+__device__ __forceinline__ bool wait_phase_poll(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                const DecodeParams &p, uint32_t backoff_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t k = 1;; ++k) {
         if (backoff_ns) __nanosleep(backoff_ns);
@@ -212,21 +212,36 @@ __device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, vol
         }
     }
 }
+__device__ __noinline__ bool wait_phase_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             const DecodeParams &p, uint32_t backoff_ns) {
+    return wait_phase_poll(bar, parity, abort_flag, p, backoff_ns);
+}
 // The MMA-issuing thread spins (backoff 0); waiting worker threads back off between
 // polls so they take few issue slots from the warps that share their scheduler.
 constexpr uint32_t kWorkerBackoffNs = 32;
+// kInline (here and in the functions below that take it): the rare paths -- the polling
+// loop of a wait that does not complete at once, the rescale of the softmax -- inline, or
+// as calls.  Measured per kernel on B200: the CTA-pair kernel runs faster with them inline
+// (B=64 x topk 512: 26.7 vs 28.0 us), the single-split kernel with calls, whose smaller
+// worker code spills less (B=256 x topk 512: 74.8 vs 76.8 us).
+template <bool kInline>
 __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                            const DecodeParams &p, uint32_t backoff_ns = 0) {
-    return mbar_test_wait(bar, parity) || wait_phase_slow(bar, parity, abort_flag, p, backoff_ns);
+    if (mbar_test_wait(bar, parity)) return true;
+    if constexpr (kInline)
+        return wait_phase_poll(bar, parity, abort_flag, p, backoff_ns);
+    else
+        return wait_phase_slow(bar, parity, abort_flag, p, backoff_ns);
 }
 
 // Warp-uniform version: lane 0 waits (acquire), the verdict is broadcast, and the warp
 // synchronisation orders the other lanes after its observation.
+template <bool kInline>
 __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                 const DecodeParams &p, int lane,
                                                 uint32_t backoff_ns = kWorkerBackoffNs) {
     int ok = 1;
-    if (lane == 0) ok = wait_phase(bar, parity, abort_flag, p, backoff_ns) ? 1 : 0;
+    if (lane == 0) ok = wait_phase<kInline>(bar, parity, abort_flag, p, backoff_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
@@ -239,11 +254,12 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
 // serialise 512 accesses to one address).  `enabled` false skips the wait but keeps
 // the barrier (every worker calls these with the same arguments).  Returns false if
 // the wait failed or was skipped.
+template <bool kInline>
 __device__ __forceinline__ bool workers_wait(uint64_t *bar, uint32_t parity, const DecodeParams &p, int t,
                                              bool enabled = true, uint32_t backoff_ns = kWorkerBackoffNs,
                                              bool failed_before = false) {
     bool ok = enabled;
-    if (t == kWaiter && enabled) ok = wait_phase(bar, parity, sm_abort(), p, backoff_ns);
+    if (t == kWaiter && enabled) ok = wait_phase<kInline>(bar, parity, sm_abort(), p, backoff_ns);
     return !barrier_or(kBarIdWorkers, kWorkers, !ok || failed_before);
 }
 
@@ -341,6 +357,7 @@ __device__ __forceinline__ void store_item(uint32_t kv, int r, int kb, int oc, b
 // i-1 has released it, and its registers then take the same dims' rows of tile i+1
 // (`next`, null for the last tile): the load issue, which stalls while the memory
 // pipeline is full, overlaps the waits for the PV instead of delaying the softmax.
+template <bool kInline>
 __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const DecodeParams &p, Slot &s,
                                              const int *next, bool &late_ok) {
     const uint32_t kv = smem_addr(g_smem + kSmemKV);
@@ -355,7 +372,7 @@ __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const Decod
     // where every worker sees it.  Fewer, larger hand-overs than one per 128-dim chunk: the
     // waits, fences and arrivals cost more than the later start of the first half.
     late_ok = true;
-    if (i > 0 && !workers_wait(&bars[kBarKvFree + 1], (i - 1) & 1, p, t)) return false;
+    if (i > 0 && !workers_wait<kInline>(&bars[kBarKvFree + 1], (i - 1) & 1, p, t)) return false;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         const int kb = 2 * c + (k8 >> 2);
@@ -376,7 +393,8 @@ __device__ __forceinline__ bool dequant_tile(int i, int t, int lane, const Decod
         load_part(0, t, next, p.cache, s);
         load_part(1, t, next, p.cache, s);
     }
-    if (i > 0) late_ok = warp_wait_phase(&bars[kBarKvFree + 3], (i - 1) & 1, sm_abort(), p, lane, 0u) && late_ok;
+    if (i > 0)
+        late_ok = warp_wait_phase<kInline>(&bars[kBarKvFree + 3], (i - 1) & 1, sm_abort(), p, lane, 0u) && late_ok;
     {
         const int kb = 4 + (k8 >> 2);
 #pragma unroll
@@ -465,6 +483,7 @@ __device__ __forceinline__ void issue_pv_wide(uint32_t d, uint32_t a_lo, uint32_
 // tile's dims chunks, then, once every worker has written P^T, O^T += V^T.P^T with a
 // commit per 128-dim chunk (freeing that chunk of the tile buffer; in the last tile it
 // makes that chunk of O^T final).
+template <bool kInline>
 __device__ __forceinline__ void mma_issue_loop(uint32_t tmem, const DecodeParams &p, int n) {
     uint64_t *bars = sm_bars();
     volatile int *abort_flag = sm_abort();
@@ -479,8 +498,8 @@ __device__ __forceinline__ void mma_issue_loop(uint32_t tmem, const DecodeParams
         const uint32_t s_col = tmem + kTmemS;
 #pragma unroll 1
         for (int cp = 0; cp < 4 && ok; ++cp) {
-            ok = (i > 0 || cp > 0 || wait_phase(&bars[kBarQ], 0, abort_flag, p)) &&
-                 wait_phase(&bars[kBarKvFull + cp], i & 1, abort_flag, p);
+            ok = (i > 0 || cp > 0 || wait_phase<kInline>(&bars[kBarQ], 0, abort_flag, p)) &&
+                 wait_phase<kInline>(&bars[kBarKvFull + cp], i & 1, abort_flag, p);
             if (!ok) break;
             tc_fence_after_sync();
             issue_qk_chunk(s_col, qk_a + cp * 2 * ((kTile * 128) >> 4), qk_b + cp * 2 * (8192 >> 4), cp == 0);
@@ -489,7 +508,7 @@ __device__ __forceinline__ void mma_issue_loop(uint32_t tmem, const DecodeParams
         const bool hook = (i == 0) && (p.debug_flags & SMLA_DEBUG_SKIP_FIRST_COMMIT);
         mma_commit(hook ? &bars[kBarSpare] : &bars[kBarSFull + (i & 1)]);
         spare_used = spare_used || hook;
-        ok = wait_phase(&bars[kBarPFull], i & 1, abort_flag, p);
+        ok = wait_phase<kInline>(&bars[kBarPFull], i & 1, abort_flag, p);
         if (!ok) break;
         tc_fence_after_sync();
 #pragma unroll 1
@@ -524,9 +543,11 @@ struct Worker {
     // kRescaleThreshold; P^T is written as bf16 hi + lo terms.  The scores are read from
     // tensor memory once; the running sums, which the PV does not read, are updated
     // after P^T has been handed to the tensor core.
+    template <bool kInline>
     __device__ __forceinline__ bool softmax(int i, bool failed_before = false) {
         // the tensor core is idle until P^T is written: wake up without backoff
-        if (!workers_wait(&sm_bars()[kBarSFull + (i & 1)], (i >> 1) & 1, p, t, true, 0u, failed_before)) return false;
+        if (!workers_wait<kInline>(&sm_bars()[kBarSFull + (i & 1)], (i >> 1) & 1, p, t, true, 0u, failed_before))
+            return false;
         tc_fence_after_sync();
         const float c = p.scale_log2;
         const bool valid = (sm_mask()[(i & 3) * 4 + q] >> lane) & 1u;
@@ -544,7 +565,10 @@ struct Worker {
             over |= (x[h] - mm[h]) > kRescaleThreshold;
         }
         if (barrier_or(kBarIdWorkers, kWorkers, over)) {
-            rescale(i, valid, s_col);
+            if constexpr (kInline)
+                rescale(i, valid, s_col);
+            else
+                rescale_call(i, valid, s_col);
             load16(hm, mm);
         }
         // p = 2^(s c - m) (0 for a masked token); P^T row r as bf16 hi + lo
@@ -585,8 +609,10 @@ struct Worker {
 
     // Raises each head's running max to max(m, tile max) and rescales what was
     // accumulated (O^T and the sums) by 2^(m_old - m_new).  Rare: the max moves only
-    // past kRescaleThreshold, and on the first tile with a valid token.
-    __device__ __noinline__ void rescale(int i, bool valid, uint32_t s_col) {
+    // past kRescaleThreshold, and on the first tile with a valid token.  rescale_call is
+    // the same as an out-of-line call.
+    __device__ __noinline__ void rescale_call(int i, bool valid, uint32_t s_col) { rescale(i, valid, s_col); }
+    __device__ __forceinline__ void rescale(int i, bool valid, uint32_t s_col) {
         const float c = p.scale_log2;
         float y[16];
         tmem_ld16(s_col, y);
@@ -663,6 +689,7 @@ __device__ __forceinline__ int slot_index(const DecodeParams &p, int t_begin, in
     return (t_begin + tile) * kTile + t;
 }
 
+template <bool kInline>
 __device__ __forceinline__ bool worker_step(Worker &w, int i, int n, int t_begin, int seq_len, const int32_t *bt_row,
                                             const int32_t *idx_row, Translator &tr, Slot &cur) {
     const DecodeParams &p = w.p;
@@ -674,8 +701,8 @@ __device__ __forceinline__ bool worker_step(Worker &w, int i, int n, int t_begin
     }
     const int *next = (i + 1 < n) ? sm_codes() + ((i + 1) & 1) * kTile : nullptr;
     bool late_ok;
-    if (!dequant_tile(i, t, w.lane, p, cur, next, late_ok)) return false;  // uniform over the workers
-    if (!w.softmax(i, !late_ok)) return false;                           // uniform too
+    if (!dequant_tile<kInline>(i, t, w.lane, p, cur, next, late_ok)) return false;  // uniform over the workers
+    if (!w.softmax<kInline>(i, !late_ok)) return false;                           // uniform too
     if (t < kTile && i + 2 < n) {
         // tile i's codes are dead (its rows were loaded one step ago): tile i+2 takes the buffer
         const int code = slot_in_range(tr.idx_a, seq_len, p.max_blocks)
@@ -744,7 +771,7 @@ __device__ __forceinline__ void write_chunk(const Worker &w, int c, const float 
 template <int kEpi>
 __device__ __forceinline__ void epilogue_direct(Worker &w, int b, int split, int n, bool ok) {
     const DecodeParams &p = w.p;
-    if (n > 0) ok = workers_wait(&sm_bars()[kBarKvFree + 3], (n - 1) & 1, p, w.t, ok);
+    if (n > 0) ok = workers_wait<false>(&sm_bars()[kBarKvFree + 3], (n - 1) & 1, p, w.t, ok);
     float *inv = sm_red();
     if (w.t < kHeads) {
         const float l = sm_head_alpha()[w.t];
@@ -797,7 +824,7 @@ __device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) 
                      "r"(__float_as_uint(lam)), "r"(bar)
                      : "memory");
     }
-    const bool got = workers_wait(&bars[kBarMl], 0, p, t);
+    const bool got = workers_wait<true>(&bars[kBarMl], 0, p, t);
     float *scale = sm_red();
     if (t < kHeads) {
         const float other = got ? sm_peer_lam()[t] : NAN;
@@ -817,7 +844,7 @@ __device__ __forceinline__ void epilogue_pair(Worker &w, int b, int n, bool ok) 
 #pragma unroll 1
     for (int k = 0; k < 4; ++k) {
         const int c = (k + 2 * me) & 3;
-        const bool chunk_ok = workers_wait(&bars[kBarKvFree + c], (n - 1) & 1, p, t, ok && n > 0);
+        const bool chunk_ok = workers_wait<true>(&bars[kBarKvFree + c], (n - 1) & 1, p, t, ok && n > 0);
         // a split without tiles adds zeros; a failed wait NaN
         const int source = chunk_ok ? kChunkTmem : (ok && n == 0) ? kChunkZero : kChunkNan;
         write_chunk<kAddF32>(w, c, sc, base, kDim, source);
@@ -938,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kCtlWarp) {
         // ================================================================ MMA issue
-        if (lane == 0 && n > 0) mma_issue_loop(tmem, p, n);
+        if (lane == 0 && n > 0) mma_issue_loop<kPair>(tmem, p, n);
         __syncwarp();
         if constexpr (kPair) cluster_wait();
     } else {
@@ -948,7 +975,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n > 0) load_slot(tid, codes, p.cache, slot);
         // tile 1's rows head for L2 right behind tile 0's (its register loads come later)
         if (tid >= kTile && tid < 2 * kTile && codes[tid] >= 0) prefetch_token_l2(p.cache, codes[tid]);
-        for (int i = 0; i < n && ok; ++i) ok = worker_step(w, i, n, t_begin, seq_len, bt_row, idx_row, tr, slot);
+        for (int i = 0; i < n && ok; ++i)
+            ok = worker_step<kPair>(w, i, n, t_begin, seq_len, bt_row, idx_row, tr, slot);
         ok = ok && !*sm_abort();
         ok = !barrier_or(kBarIdWorkers, kWorkers, !ok);
         w.reduce_sums(ok && n > 0);
